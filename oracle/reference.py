@@ -1,0 +1,239 @@
+"""Plain float64 definitions of what the decode step computes (oracle).
+
+TEST INFRASTRUCTURE ONLY -- see the package docstring.
+
+Everything here is the mathematical definition evaluated in float64 from the
+fp32 inputs: no blocking, no splitting, no fixed-split softmax.  The fixed
+reduction orders of the batch-invariant kernels [BI] are GPU strategies for
+reproducing *one* rounding of these definitions; the oracle instead computes
+the exact-as-possible value the method approximates.  The only encodings used
+are the KV-cache quantiser (the cache is INT16 by definition [HEAL, section
+"1. 「スマート・パッキング」のトリック"]) from `oracle.encodings`.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+from . import encodings as enc
+
+
+def f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+# ----------------------------------------------------------------------------
+# matrix product  [HEAL, section "2. 「誤差補償」のトリック（計算用）": the
+# compensated GEMM targets FP32-grade accuracy of y = x W]
+# ----------------------------------------------------------------------------
+
+def gemm(A, W) -> np.ndarray:
+    """y = A W in float64 (fp32 products are exact in float64)."""
+    return f64(A) @ f64(W)
+
+
+def gemm_fp16_only(A, W) -> np.ndarray:
+    """Diagnostic: the uncompensated 16-bit product rn16(A) rn16(W), float64 sums."""
+    a = enc.f16_bits_to_f64(enc.rn16_bits(f64(np.asarray(A, np.float32))))
+    w = enc.f16_bits_to_f64(enc.rn16_bits(f64(np.asarray(W, np.float32))))
+    return a @ w
+
+
+def gemm_split3(A, W) -> np.ndarray:
+    """Diagnostic: the three-product algebra A_hi B_hi + 2^-11 (A_hi B_lo + A_lo B_hi),
+    rescaled by 2^-e_n, summed in float64 (isolates truncation from rounding)."""
+    a_hi, a_lo, _ = enc.heal_split(A, 0)
+    e = enc.column_exponents(W).astype(np.int64)
+    w_hi, w_lo, _ = enc.heal_split(W, e[None, :])
+    ah, al = enc.f16_bits_to_f64(a_hi), enc.f16_bits_to_f64(a_lo)
+    wh, wl = enc.f16_bits_to_f64(w_hi), enc.f16_bits_to_f64(w_lo)
+    y = ah @ wh + np.ldexp(ah @ wl + al @ wh, -enc.LO_SCALE_LOG2)
+    return np.ldexp(y, -e[None, :])
+
+
+# ----------------------------------------------------------------------------
+# RMSNorm  [BI, table row "RMSNorm"]
+# ----------------------------------------------------------------------------
+
+def rmsnorm(x, gamma, eps) -> np.ndarray:
+    """y = x / sqrt(mean(x^2) + eps) * gamma, per row, float64."""
+    x = f64(x)
+    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + float(eps))
+    return x * r * f64(gamma)
+
+
+# ----------------------------------------------------------------------------
+# rotary position embedding (rotate-half pairing (i, i + D/2), theta_i = base^(-2i/D))
+# ----------------------------------------------------------------------------
+
+def rope_angles(pos, head_dim: int, base: float = 10000.0) -> np.ndarray:
+    """angle[p, i] = pos_p * base^(-2 i / D), float64 [len(pos), D/2]."""
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    theta = np.power(float(base), -2.0 * i / head_dim)
+    return f64(pos)[:, None] * theta[None, :]
+
+
+def apply_rope(x, pos, base: float = 10000.0) -> np.ndarray:
+    """Rotate x[T, H, D] by the angles of positions pos[T] (float64)."""
+    x = f64(x)
+    D = x.shape[-1]
+    ang = rope_angles(pos, D, base)[:, None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = x[..., : D // 2], x[..., D // 2:]
+    return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+
+
+# ----------------------------------------------------------------------------
+# KV cache (INT16 codes + fp32 scales, layout [slot][kv_head][pos][D])
+# ----------------------------------------------------------------------------
+
+@dataclass
+class KVCache:
+    k: np.ndarray        # int16 [S, Hkv, Lmax, D]
+    ks: np.ndarray       # fp32  [S, Hkv, Lmax]
+    v: np.ndarray
+    vs: np.ndarray
+
+    @staticmethod
+    def empty(n_slots: int, n_kv: int, max_len: int, head_dim: int) -> "KVCache":
+        return KVCache(np.zeros((n_slots, n_kv, max_len, head_dim), np.int16),
+                       np.zeros((n_slots, n_kv, max_len), np.float32),
+                       np.zeros((n_slots, n_kv, max_len, head_dim), np.int16),
+                       np.zeros((n_slots, n_kv, max_len), np.float32))
+
+    def write(self, which: str, x, slot, pos) -> None:
+        """Quantise fp32 x[T, Hkv, D] and store it at (slot[t], :, pos[t])."""
+        q, s = enc.kv_quant_int16(np.asarray(x, np.float32))
+        codes, scales = (self.k, self.ks) if which == "k" else (self.v, self.vs)
+        for t in range(q.shape[0]):
+            codes[slot[t], :, pos[t]] = q[t]
+            scales[slot[t], :, pos[t]] = s[t]
+
+
+# ----------------------------------------------------------------------------
+# decode attention over the dequantised cache  [BI, table row "Attention";
+# HEAL, section "1. 「スマート・パッキング」のトリック"]
+# ----------------------------------------------------------------------------
+
+def attention_decode(q, cache: KVCache, slot, length, softmax_scale, return_probs=False):
+    """One query row per sequence: out[b, h] = sum_j p_j V~_j with
+    p = softmax_j(sigma q_h . K~_j) over the first length[b] keys of slot[b].
+
+    q: [B, Hq, D]; K~/V~ are the exact float64 dequantised cache values; query
+    head h reads kv head h // (Hq / Hkv).  softmax_scale is taken as the fp32
+    value the caller passes, promoted to float64.  The softmax is one pass over
+    all keys (the definition), not the GPU's fixed 256-key splits.
+    """
+    q = f64(q)
+    B, Hq, D = q.shape
+    Hkv = cache.k.shape[1]
+    G = Hq // Hkv
+    sigma = float(np.float32(softmax_scale))
+    out = np.zeros((B, Hq, D), np.float64)
+    probs = []
+    for b in range(B):
+        L = int(length[b])
+        s = int(slot[b])
+        Kt = enc.kv_dequant(cache.k[s, :, :L], cache.ks[s, :, :L])   # [Hkv, L, D]
+        Vt = enc.kv_dequant(cache.v[s, :, :L], cache.vs[s, :, :L])
+        qb = q[b].reshape(Hkv, G, D)
+        t = sigma * np.einsum("hgd,hld->hgl", qb, Kt)                # [Hkv, G, L]
+        t = t - t.max(axis=-1, keepdims=True)
+        p = np.exp(t)
+        p = p / p.sum(axis=-1, keepdims=True)
+        out[b] = np.einsum("hgl,hld->hgd", p, Vt).reshape(Hq, D)
+        if return_probs:
+            probs.append(p.reshape(Hq, L))
+    return (out, probs) if return_probs else out
+
+
+# ----------------------------------------------------------------------------
+# decode layer and layer stack (LLaMA-style block: RMSNorm -> GQA attention with
+# rotary embedding over the INT16 cache -> residual -> RMSNorm -> SwiGLU MLP ->
+# residual)
+# ----------------------------------------------------------------------------
+
+@dataclass
+class LayerParams:
+    wq: np.ndarray        # fp32 [H, Hq*D]
+    wk: np.ndarray        # fp32 [H, Hkv*D]
+    wv: np.ndarray        # fp32 [H, Hkv*D]
+    wo: np.ndarray        # fp32 [Hq*D, H]
+    w_gate: np.ndarray    # fp32 [H, F]
+    w_up: np.ndarray      # fp32 [H, F]
+    w_down: np.ndarray    # fp32 [F, H]
+    g_attn: np.ndarray    # fp32 [H]
+    g_mlp: np.ndarray     # fp32 [H]
+    n_heads: int
+    n_kv_heads: int
+    head_dim: int
+    eps: float = 1e-6
+    rope_base: float = 10000.0
+
+
+def silu(x) -> np.ndarray:
+    x = f64(x)
+    return x / (1.0 + np.exp(-x))
+
+
+def decode_layer(p: LayerParams, cache: KVCache, x, slot, pos, softmax_scale=None,
+                 return_intermediates=False):
+    """One layer over B token rows; row b belongs to cache slot slot[b] at position
+    pos[b].  The K/V of every row are quantised into the cache before any row
+    attends, and row b attends over positions 0..pos[b] of its slot.  Returns the
+    float64 output rows (and optionally the intermediates)."""
+    x = f64(np.asarray(x, np.float32))
+    B = x.shape[0]
+    Hq, Hkv, D = p.n_heads, p.n_kv_heads, p.head_dim
+    sigma = np.float32(1.0 / np.sqrt(D)) if softmax_scale is None else np.float32(softmax_scale)
+    slot = np.asarray(slot, np.int64)
+    pos = np.asarray(pos, np.int64)
+
+    h = rmsnorm(x, p.g_attn, p.eps)
+    q = (h @ f64(p.wq)).reshape(B, Hq, D)
+    k = (h @ f64(p.wk)).reshape(B, Hkv, D)
+    v = (h @ f64(p.wv)).reshape(B, Hkv, D)
+    q = apply_rope(q, pos, p.rope_base)
+    k = apply_rope(k, pos, p.rope_base)
+    cache.write("k", k.astype(np.float32), slot, pos)
+    cache.write("v", v.astype(np.float32), slot, pos)
+    o = attention_decode(q, cache, slot, pos + 1, sigma).reshape(B, Hq * D)
+    x1 = x + o @ f64(p.wo)
+    h2 = rmsnorm(x1, p.g_mlp, p.eps)
+    a = silu(h2 @ f64(p.w_gate)) * (h2 @ f64(p.w_up))
+    out = x1 + a @ f64(p.w_down)
+    if return_intermediates:
+        return out, dict(h=h, q=q, k=k, v=v, o=o, x1=x1, h2=h2, a=a)
+    return out
+
+
+@dataclass
+class StackParams:
+    embed: np.ndarray      # fp32 [V, H]
+    layers: list           # [LayerParams]
+    g_final: np.ndarray    # fp32 [H]
+    lm_head: np.ndarray    # fp32 [H, V]
+    eps: float = 1e-6
+
+
+def argmax_lowest(logits) -> np.ndarray:
+    """Index of the maximum per row; ties go to the lowest index (np.argmax)."""
+    return np.argmax(f64(logits), axis=-1).astype(np.int64)
+
+
+def stack_forward(sp: StackParams, caches, tokens, slot, pos, return_hidden=False):
+    """Token ids -> embedding -> every layer -> final RMSNorm -> LM head ->
+    (logits, greedy ids).  Hidden states between layers are rounded to fp32,
+    the container every inter-layer tensor uses."""
+    x = np.asarray(sp.embed, np.float32)[np.asarray(tokens, np.int64)]
+    hidden = []
+    for li, lp in enumerate(sp.layers):
+        x = decode_layer(lp, caches[li], x, slot, pos).astype(np.float32)
+        hidden.append(x)
+    hf = rmsnorm(x, sp.g_final, sp.eps)
+    logits = hf @ f64(sp.lm_head)
+    ids = argmax_lowest(logits)
+    if return_hidden:
+        return logits, ids, hidden
+    return logits, ids

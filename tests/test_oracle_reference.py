@@ -1,0 +1,281 @@
+"""Pins for the oracle's float64 reference definitions (CPU only).
+
+Checked against exact rational arithmetic, closed forms, invariants and
+independent library implementations (torch's rms_norm and scaled-dot-product
+attention, the Hugging Face LLaMA decoder block and model).
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from invariant_numerics_b200 import synth
+from oracle import encodings as enc
+from oracle import reference as ref
+
+
+# ---------------------------------------------------------------- GEMM --------
+
+def test_gemm_brute_force_rational():
+    A = synth.normal((3, 7), seed=1)
+    W = synth.normal((7, 5), seed=2, std=0.02)
+    y = ref.gemm(A, W)
+    for m in range(3):
+        for n in range(5):
+            exact = sum(Fraction(float(A[m, k])) * Fraction(float(W[k, n])) for k in range(7))
+            bound = sum(abs(float(A[m, k]) * float(W[k, n])) for k in range(7)) * 7 * 2.0**-52
+            assert abs(float(Fraction(y[m, n]) - exact)) <= bound
+
+
+def test_gemm_dyadic_inputs_exact():
+    # small dyadic rationals: every product and partial sum is exact in float64
+    g = np.random.Generator(np.random.PCG64(5))
+    A = (g.integers(-64, 64, size=(4, 8)) / 8.0).astype(np.float32)
+    W = (g.integers(-64, 64, size=(8, 6)) / 16.0).astype(np.float32)
+    y = ref.gemm(A, W)
+    for m in range(4):
+        for n in range(6):
+            exact = sum(Fraction(float(A[m, k])) * Fraction(float(W[k, n])) for k in range(8))
+            assert Fraction(y[m, n]) == exact
+
+
+def test_split3_identity_weight_is_reconstruction():
+    A = synth.normal_with_outliers((5, 64), seed=3)
+    W = np.eye(64, dtype=np.float32)
+    y = ref.gemm_split3(A, W)
+    hi, lo, _ = enc.heal_split(A)
+    assert np.array_equal(y, enc.heal_reconstruct(hi, lo))
+
+
+def test_split3_fp16_exact_inputs_equal_fp16_product():
+    g = np.random.Generator(np.random.PCG64(6))
+    A = g.integers(-100, 100, size=(3, 16)).astype(np.float32)
+    W = g.integers(-100, 100, size=(16, 64)).astype(np.float32)
+    assert np.array_equal(ref.gemm_split3(A, W), ref.gemm(A, W))
+    assert np.array_equal(ref.gemm_fp16_only(A, W), ref.gemm(A, W))
+
+
+def test_compensated_error_far_below_fp16_only():
+    # the GEMM sweep's input model: N(0,1) activations with 0.1% outliers x100,
+    # N(0, 0.02) weights
+    A = synth.normal_with_outliers((16, 1024), seed=9)
+    W = synth.normal((1024, 128), seed=10, std=0.02)
+    y = ref.gemm(A, W)
+    e3 = np.abs(ref.gemm_split3(A, W) - y).max()
+    e16 = np.abs(ref.gemm_fp16_only(A, W) - y).max()
+    scale = np.abs(y).max()
+    assert e3 <= 1e-6 * scale
+    assert e3 <= 1e-2 * e16
+    # truncation error of the three-product algebra obeys its per-product bound
+    bound = (np.abs(A).astype(np.float64) @ np.abs(W).astype(np.float64)) * 3 * 2.0**-22
+    assert (np.abs(ref.gemm_split3(A, W) - y) <= bound).all()
+
+
+# ------------------------------------------------------------- RMSNorm --------
+
+def test_rmsnorm_constant_row_closed_form():
+    for c in (3.0, -0.5, 1e-4):
+        x = np.full((1, 512), c, np.float32)
+        gamma = synth.uniform(512, seed=4, lo=0.5, hi=1.5)
+        y = ref.rmsnorm(x, gamma, 1e-6)
+        want = gamma.astype(np.float64) * np.float64(np.float32(c)) / np.sqrt(np.float64(np.float32(c)) ** 2 + 1e-6)
+        np.testing.assert_allclose(y[0], want, rtol=1e-14, atol=0)
+
+
+def test_rmsnorm_matches_torch():
+    x = synth.normal((7, 4096), seed=5)
+    gamma = synth.uniform(4096, seed=6, lo=0.5, hi=1.5)
+    y = ref.rmsnorm(x, gamma, 1e-6)
+    yt = torch.nn.functional.rms_norm(torch.from_numpy(x).double(), (4096,),
+                                      torch.from_numpy(gamma).double(), eps=1e-6)
+    np.testing.assert_allclose(y, yt.numpy(), rtol=1e-13, atol=0)
+
+
+# ---------------------------------------------------------------- RoPE --------
+
+def test_rope_identity_at_zero_and_norm_preserving():
+    x = synth.normal((3, 4, 128), seed=7)
+    np.testing.assert_array_equal(ref.apply_rope(x, [0, 0, 0]), x.astype(np.float64))
+    y = ref.apply_rope(x, [5, 100, 4000])
+    a, b = x[..., :64].astype(np.float64), x[..., 64:].astype(np.float64)
+    ya, yb = y[..., :64], y[..., 64:]
+    np.testing.assert_allclose(ya**2 + yb**2, a**2 + b**2, rtol=1e-12)
+
+
+def test_rope_matches_hf_llama():
+    from transformers.models.llama.modeling_llama import apply_rotary_pos_emb
+    x = synth.normal((1, 2, 6, 128), seed=8).astype(np.float64)       # [b, h, t, d]
+    pos = np.array([0, 1, 2, 7, 33, 101])
+    ang = ref.rope_angles(pos, 128)
+    cos = torch.from_numpy(np.concatenate([np.cos(ang)] * 2, axis=-1))[None]
+    sin = torch.from_numpy(np.concatenate([np.sin(ang)] * 2, axis=-1))[None]
+    q_hf, _ = apply_rotary_pos_emb(torch.from_numpy(x), torch.from_numpy(x), cos, sin)
+    ours = ref.apply_rope(np.transpose(x[0], (1, 0, 2)), pos)           # [t, h, d]
+    np.testing.assert_allclose(np.transpose(ours, (1, 0, 2)), q_hf[0].numpy(), rtol=0, atol=1e-13)
+
+
+# ----------------------------------------------------------- attention --------
+
+def _cache_with(k, v, n_slots=None):
+    """k, v fp32 [B, Hkv, L, D] -> oracle cache with one slot per row."""
+    B, Hkv, L, D = k.shape
+    c = ref.KVCache.empty(B if n_slots is None else n_slots, Hkv, L, D)
+    for b in range(B):
+        for p in range(L):
+            c.write("k", k[b:b + 1, :, p], [b], [p])
+            c.write("v", v[b:b + 1, :, p], [b], [p])
+    return c
+
+
+def test_attention_probabilities_sum_to_one_and_match_sdpa():
+    B, Hq, Hkv, L, D = 2, 8, 2, 37, 128
+    k = synth.kv_tensor(B * L, Hkv, D, seed=1).reshape(B, L, Hkv, D).transpose(0, 2, 1, 3).copy()
+    v = synth.kv_tensor(B * L, Hkv, D, seed=2).reshape(B, L, Hkv, D).transpose(0, 2, 1, 3).copy()
+    cache = _cache_with(k, v)
+    q = synth.normal((B, Hq, D), seed=3)
+    lens = np.array([37, 20])
+    sigma = np.float32(1 / np.sqrt(128))
+    out, probs = ref.attention_decode(q, cache, [0, 1], lens, sigma, return_probs=True)
+    for p in probs:
+        assert np.abs(p.sum(axis=-1) - 1).max() <= 1e-12
+    for b in range(B):
+        Lb = lens[b]
+        Kd = enc.kv_dequant(cache.k[b, :, :Lb], cache.ks[b, :, :Lb])
+        Vd = enc.kv_dequant(cache.v[b, :, :Lb], cache.vs[b, :, :Lb])
+        qt = torch.from_numpy(q[b].astype(np.float64))[None, :, None, :]       # [1, Hq, 1, D]
+        Kt = torch.from_numpy(np.repeat(Kd, Hq // Hkv, axis=0))[None]           # [1, Hq, L, D]
+        Vt = torch.from_numpy(np.repeat(Vd, Hq // Hkv, axis=0))[None]
+        o = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, scale=float(sigma))
+        np.testing.assert_allclose(out[b], o[0, :, 0].numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_attention_single_key_and_equal_keys():
+    Hq, Hkv, D = 4, 1, 128
+    k = synth.kv_tensor(1, Hkv, D, seed=4)[None].transpose(0, 2, 1, 3).copy()   # [1, 1, 1, D]
+    v = synth.kv_tensor(5, Hkv, D, seed=5).reshape(1, 5, Hkv, D).transpose(0, 2, 1, 3).copy()
+    kk = np.repeat(k, 5, axis=2)
+    cache = _cache_with(kk, v)
+    q = synth.normal((1, Hq, D), seed=6)
+    # one key: the output is exactly the dequantised value row
+    o1 = ref.attention_decode(q, cache, [0], [1], 0.125)
+    Vd = enc.kv_dequant(cache.v[0, :, :5], cache.vs[0, :, :5])
+    for h in range(Hq):
+        np.testing.assert_array_equal(o1[0, h], Vd[0, 0])
+    # five identical keys: uniform probabilities, output = mean of the values
+    o5 = ref.attention_decode(q, cache, [0], [5], 0.125)
+    for h in range(Hq):
+        np.testing.assert_allclose(o5[0, h], Vd[0].mean(axis=0), rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------- layer and stack --------
+
+def _small_layer(seed=0, H=128, Hq=4, Hkv=2, D=32, F=256):
+    s = lambda i, shape, std=0.02: synth.normal(shape, seed=seed, stream=i, std=std)
+    return ref.LayerParams(
+        wq=s(1, (H, Hq * D), 0.08), wk=s(2, (H, Hkv * D), 0.08), wv=s(3, (H, Hkv * D), 0.08),
+        wo=s(4, (Hq * D, H), 0.08), w_gate=s(5, (H, F), 0.08), w_up=s(6, (H, F), 0.08),
+        w_down=s(7, (F, H), 0.08),
+        g_attn=synth.uniform(H, seed=seed, stream=8, lo=0.5, hi=1.5),
+        g_mlp=synth.uniform(H, seed=seed, stream=9, lo=0.5, hi=1.5),
+        n_heads=Hq, n_kv_heads=Hkv, head_dim=D)
+
+
+def _hf_config(p, H, F, V=64, layers=1):
+    from transformers import LlamaConfig
+    cfg = LlamaConfig(vocab_size=V, hidden_size=H, intermediate_size=F, num_hidden_layers=layers,
+                      num_attention_heads=p.n_heads, num_key_value_heads=p.n_kv_heads,
+                      head_dim=p.head_dim, rms_norm_eps=p.eps, rope_theta=p.rope_base,
+                      max_position_embeddings=4096, attention_bias=False, mlp_bias=False,
+                      tie_word_embeddings=False)
+    cfg._attn_implementation = "eager"
+    return cfg
+
+
+def _load_hf_layer(layer, p):
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a.astype(np.float64).T))
+    with torch.no_grad():
+        layer.self_attn.q_proj.weight.copy_(t(p.wq))
+        layer.self_attn.k_proj.weight.copy_(t(p.wk))
+        layer.self_attn.v_proj.weight.copy_(t(p.wv))
+        layer.self_attn.o_proj.weight.copy_(t(p.wo))
+        layer.mlp.gate_proj.weight.copy_(t(p.w_gate))
+        layer.mlp.up_proj.weight.copy_(t(p.w_up))
+        layer.mlp.down_proj.weight.copy_(t(p.w_down))
+        layer.input_layernorm.weight.copy_(torch.from_numpy(p.g_attn.astype(np.float64)))
+        layer.post_attention_layernorm.weight.copy_(torch.from_numpy(p.g_mlp.astype(np.float64)))
+
+
+def test_decode_layer_prefill_matches_hf_llama_block():
+    """Causal prefill of one sequence through the oracle layer (INT16 cache)
+    against the Hugging Face LLaMA model with one layer (float cache)."""
+    from transformers import LlamaModel
+    H, F, T = 128, 256, 24
+    p = _small_layer(seed=1, H=H, F=F)
+    cfg = _hf_config(p, H, F)
+    model = LlamaModel(cfg).double().eval()
+    _load_hf_layer(model.layers[0], p)
+    x = synth.normal((T, H), seed=2)
+    cache = ref.KVCache.empty(1, p.n_kv_heads, 64, p.head_dim)
+    ours = ref.decode_layer(p, cache, x, np.zeros(T, np.int64), np.arange(T))
+    captured = {}
+
+    def hook(mod, args, output):
+        captured["y"] = output[0] if isinstance(output, tuple) else output
+
+    handle = model.layers[0].register_forward_hook(hook)
+    with torch.no_grad():
+        model(inputs_embeds=torch.from_numpy(x.astype(np.float64))[None])
+    handle.remove()
+    hf = captured["y"][0].numpy()          # output of the block, before the final norm
+    err = np.abs(ours - hf).max(axis=1) / np.abs(hf).max(axis=1)
+    assert err.max() < 2e-4, err.max()     # INT16 cache vs float cache
+    # chunked prefill through the oracle gives the same rows as one shot
+    cache2 = ref.KVCache.empty(1, p.n_kv_heads, 64, p.head_dim)
+    parts = [ref.decode_layer(p, cache2, x[a:b], np.zeros(b - a, np.int64), np.arange(a, b))
+             for a, b in ((0, 7), (7, 8), (8, 24))]
+    # (float64 BLAS itself varies its blocking with the row count, so this
+    # semantic check of chunking uses a tolerance rather than bit identity)
+    np.testing.assert_allclose(np.concatenate(parts), ours, rtol=1e-12, atol=1e-12)
+
+
+def test_decode_layer_zero_projections_is_identity():
+    p = _small_layer(seed=3)
+    p.wo[:] = 0
+    p.w_down[:] = 0
+    x = synth.normal((5, 128), seed=4)
+    cache = ref.KVCache.empty(5, p.n_kv_heads, 8, p.head_dim)
+    out = ref.decode_layer(p, cache, x, np.arange(5), np.full(5, 3))
+    np.testing.assert_array_equal(out, x.astype(np.float64))
+
+
+def test_stack_matches_hf_llama_causal_lm():
+    from transformers import LlamaForCausalLM
+    H, F, V, T, nl = 128, 256, 96, 16, 2
+    layers = [_small_layer(seed=10 + i, H=H, F=F) for i in range(nl)]
+    sp = ref.StackParams(embed=synth.normal((V, H), seed=20), layers=layers,
+                         g_final=synth.uniform(H, seed=21, lo=0.5, hi=1.5),
+                         lm_head=synth.normal((H, V), seed=22, std=0.08))
+    cfg = _hf_config(layers[0], H, F, V=V, layers=nl)
+    model = LlamaForCausalLM(cfg).double().eval()
+    with torch.no_grad():
+        model.model.embed_tokens.weight.copy_(torch.from_numpy(sp.embed.astype(np.float64)))
+        model.model.norm.weight.copy_(torch.from_numpy(sp.g_final.astype(np.float64)))
+        model.lm_head.weight.copy_(torch.from_numpy(np.ascontiguousarray(sp.lm_head.astype(np.float64).T)))
+        for i in range(nl):
+            _load_hf_layer(model.model.layers[i], layers[i])
+    tokens = synth.token_ids(T, V, seed=23)
+    caches = [ref.KVCache.empty(1, 2, 32, 32) for _ in range(nl)]
+    logits, ids = ref.stack_forward(sp, caches, tokens, np.zeros(T, np.int64), np.arange(T))
+    with torch.no_grad():
+        hf = model(input_ids=torch.from_numpy(tokens.astype(np.int64))[None]).logits[0].numpy()
+    err = np.abs(logits - hf).max(axis=1) / np.abs(hf).max(axis=1)
+    assert err.max() < 2e-4, err.max()
+    margin = np.sort(hf, axis=1)
+    clear = (margin[:, -1] - margin[:, -2]) > 1e-2 * np.abs(hf).max(axis=1)
+    assert np.array_equal(ids[clear], np.argmax(hf, axis=1)[clear])
+
+
+def test_argmax_ties_lowest_index():
+    x = np.array([[1.0, 3.0, 3.0, 2.0], [0.0, 0.0, 0.0, 0.0]])
+    assert ref.argmax_lowest(x).tolist() == [1, 0]
