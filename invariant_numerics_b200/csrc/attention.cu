@@ -1,0 +1,471 @@
+// Batch-invariant decode attention over the INT16 KV cache.
+//
+// "Defeating Nondeterminism" summary, table row Attention: one unified cache
+// layout and FIXED-SIZE splits, so a row's reduction never depends on batch
+// size, sequence length beyond its own, or prefill/decode chunking.  Splits are
+// 256 keys at absolute positions [256 s, 256 s + 256).
+// HEAL explainer, section "1. 「スマート・パッキング」のトリック": the INT16 codes
+// are unpacked into two 16-bit values for the arithmetic.  Here a code is
+// q = 256 h + l (h the signed high byte, l the low byte); h and l/256 are
+// exact binary16 numbers, so two 16-bit tensor-core products recover q/256
+// exactly before fp32 accumulation.
+//
+// Split kernel: one CTA (4 warps) per (row b, kv head, split s).  The 256 x 128
+// K codes arrive by TMA (2-D, 128-byte swizzle) into 64 KB of shared memory;
+// every warp owns 64 keys.  Scores S^T = K Q^T use mma.m16n8k16 with the 16
+// keys of an m-tile as rows and the 8 columns [q_hi, q_lo] x 4 query heads of
+// the GQA group (q split like heal_split) as N.  The split max, exp, sum and
+// a per-(split, head) power-of-two scaling of w = p s_V follow; the V codes
+// then overwrite the K buffer and O^T = V^T W runs with d as rows and
+// [w_hi, w_lo] x 4 heads as columns.  Warps' partial sums are added in warp
+// order.  Output per (row, head, split): (m, l, o[128]).
+// Combine kernel: one warp per (row, head) folds the splits s = 0, 1, ... in
+// order, o / l, and writes fp32 plus the binary16 hi/lo split.
+//
+// This is a bandwidth-bound kernel (520 bytes of codes and scales per key and
+// kv head); the warp-level MMAs only keep the 16-bit products exact at the
+// rate HBM delivers the codes.
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+using inv::record_status;
+
+constexpr int SPLIT = INV_KV_SPLIT;          // 256
+constexpr int THREADS = 128;                 // 4 warps x 64 keys
+constexpr int BOX_BYTES = 64 * 64 * 2;       // 64 keys x 64 d x int16
+constexpr int CODE_BYTES = 8 * BOX_BYTES;    // 256 keys x 128 d
+
+struct __align__(1024) AttnSmem {
+  uint8_t codes[CODE_BYTES];   // K codes, then V codes, then the warp exchange of O
+  float ks[SPLIT];
+  float vs[SPLIT];
+  float red_m[4][4];
+  float red_l[4][4];
+  float red_w[4][4];
+  uint64_t bar_k, bar_v;
+  int abort;
+};
+constexpr size_t kAttnSmem = sizeof(AttnSmem) + 1024;
+
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// Dual-FP16 unpack of two INT16 codes (low half = first).  Returns the pair of
+// high bytes h as binary16 and the pair of low bytes as l/256 in binary16:
+// (1024 + (h + 128)) - 1152 = h and (4 + l/256) - 4 = l/256, all exact.
+__device__ __forceinline__ void unpack_dual(uint32_t x, uint32_t& hpart, uint32_t& lpart) {
+  const uint32_t xs = x ^ 0x80008000u;  // biased high byte h + 128; low byte unchanged
+  const uint32_t hb = __byte_perm(xs, 0x64646464u, 0x4341);
+  const uint32_t lb = __byte_perm(xs, 0x44444444u, 0x4240);
+  const __half2 hv = __hsub2(*reinterpret_cast<const __half2*>(&hb), __halves2half2(__ushort_as_half(0x6480),
+                                                                                     __ushort_as_half(0x6480)));
+  const __half2 lv = __hsub2(*reinterpret_cast<const __half2*>(&lb), __halves2half2(__ushort_as_half(0x4400),
+                                                                                     __ushort_as_half(0x4400)));
+  hpart = *reinterpret_cast<const uint32_t*>(&hv);
+  lpart = *reinterpret_cast<const uint32_t*>(&lv);
+}
+
+// Shared address of code (key kk of the split, d0 multiple of 8) in the
+// 128-byte-swizzled TMA layout: box kk/64, d half d0/64, row kk%64, 16-byte
+// chunk ((d0%64)/8) xor (row%8).
+__device__ __forceinline__ uint32_t code_addr(uint32_t base, int kk, int d0) {
+  const int r = kk & 63;
+  return base + (kk >> 6) * (2 * BOX_BYTES) + (d0 >> 6) * BOX_BYTES + r * 128 +
+         ((((d0 & 63) >> 3) ^ (r & 7)) << 4);
+}
+
+__device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
+  return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+}
+
+__global__ void __launch_bounds__(THREADS, 3)
+    attn_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                      const float* __restrict__ q, const float* __restrict__ kscale, const float* __restrict__ vscale,
+                      const int32_t* __restrict__ slot, const int32_t* __restrict__ len, int Hq, int Hkv,
+                      int n_slots, int max_len, int len_limit, int S_max, float sigma, float* __restrict__ part_o,
+                      float2* __restrict__ part_ml, int* status, long long wait_ns) {
+  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int G = Hq / Hkv;
+  const int L = len[b], sl = slot[b];
+  if (L < 1 || L > len_limit || sl < 0 || sl >= n_slots) {
+    if (s == 0 && h == 0 && threadIdx.x == 0) record_status(status, INV_ERR_INVALID_ARG);
+    return;
+  }
+  const int key0 = s * SPLIT;
+  if (key0 >= L) return;
+  const int n = min(SPLIT, L - key0);
+  const int nbox = (n + 63) >> 6;
+  const int row0 = (int)(((int64_t)sl * Hkv + h) * max_len + key0);
+
+  extern __shared__ uint8_t smem_raw[];
+  AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
+  const uint32_t cbase = inv::smem_u32(sm.codes);
+
+  if (tid == 0) {
+    inv::mbar_init(&sm.bar_k, 1);
+    inv::mbar_init(&sm.bar_v, 1);
+    sm.abort = 0;
+    inv::fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    inv::mbar_arrive_expect_tx(&sm.bar_k, nbox * 2 * BOX_BYTES);
+    for (int bx = 0; bx < nbox; ++bx) {
+      inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES, &tm_k, &sm.bar_k, 0, row0 + 64 * bx);
+      inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES + BOX_BYTES, &tm_k, &sm.bar_k, 64, row0 + 64 * bx);
+    }
+  }
+  for (int j = tid; j < SPLIT; j += THREADS) {
+    sm.ks[j] = j < n ? kscale[(int64_t)row0 + j] : 0.0f;
+    sm.vs[j] = j < n ? vscale[(int64_t)row0 + j] : 0.0f;
+  }
+
+  // B fragments of S^T = K Q^T: column g is query head g/2 of the group, its
+  // hi part for even g and lo part for odd g; rows k = d.
+  uint32_t qf[8][2];
+  {
+    const int head = g >> 1;
+    const bool lo = (g & 1) != 0;
+    const bool valid = head < G;
+    const float* qh = q + ((int64_t)b * Hq + (int64_t)h * G + head) * 128;
+    bool bad = false;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int d = 16 * ks + 2 * c + 8 * r;
+        const float x0 = valid ? qh[d] : 0.0f, x1 = valid ? qh[d + 1] : 0.0f;
+        __half h0, l0, h1, l1;
+        inv::split_hi_lo(x0, h0, l0);
+        inv::split_hi_lo(x1, h1, l1);
+        bad |= inv::f16_overflow(x0) | inv::f16_overflow(x1);
+        qf[ks][r] = lo ? pack_half2(l0, l1) : pack_half2(h0, h1);
+      }
+    }
+    if (bad) record_status(status, INV_ERR_RANGE);
+  }
+  __syncthreads();  // scales visible
+
+  bool ok = true;
+  if (lane == 0) ok = inv::mbar_wait(&sm.bar_k, 0, wait_ns, &sm.abort, status);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+
+  // ---------------------------------------------------------------- scores --
+  float tsc[4][2];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    const int kb = warp * 64 + mt * 16;
+    tsc[mt][0] = tsc[mt][1] = -INFINITY;
+    if (ok && kb < n) {
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      const int lkey = kb + ((lane >> 3) & 1) * 8 + (lane & 7);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t a[4], ah[4], al[4];
+        ldsm_x4(code_addr(cbase, lkey, 16 * ks + (lane >> 4) * 8), a);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) unpack_dual(a[i], ah[i], al[i]);
+        mma16816(acc, ah, qf[ks][0], qf[ks][1]);
+        mma16816(acc, al, qf[ks][0], qf[ks][1]);
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int key = kb + g + 8 * r;
+        // acc[2r] = q_hi . code / 256, acc[2r+1] = q_lo . code / 256 (head c)
+        const float dot = __fmul_rn(__fadd_rn(acc[2 * r], __fmul_rn(acc[2 * r + 1], 0x1p-11f)), 256.0f);
+        const float t = __fmul_rn(__fmul_rn(dot, sm.ks[key]), sigma);
+        tsc[mt][r] = key < n ? t : -INFINITY;
+        mx = fmaxf(mx, tsc[mt][r]);
+      }
+    }
+  }
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+  if (g == 0) sm.red_m[warp][c] = mx;
+  inv::fence_proxy_async_smem();  // K reads (generic proxy) before the TMA overwrite (async proxy)
+  __syncthreads();
+
+  bool v_issued = false;
+  if (tid == 0 && ok) {
+    v_issued = true;
+    inv::mbar_arrive_expect_tx(&sm.bar_v, nbox * 2 * BOX_BYTES);
+    for (int bx = 0; bx < nbox; ++bx) {
+      inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES, &tm_v, &sm.bar_v, 0, row0 + 64 * bx);
+      inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES + BOX_BYTES, &tm_v, &sm.bar_v, 64, row0 + 64 * bx);
+    }
+  }
+
+  // ---------------------------------------------------------------- softmax --
+  const float M = fmaxf(fmaxf(sm.red_m[0][c], sm.red_m[1][c]), fmaxf(sm.red_m[2][c], sm.red_m[3][c]));
+  float w[4][2];
+  float lsum = 0.0f, wmax = 0.0f;
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int key = warp * 64 + mt * 16 + g + 8 * r;
+      const float p = tsc[mt][r] == -INFINITY ? 0.0f : expf(__fsub_rn(tsc[mt][r], M));
+      lsum = __fadd_rn(lsum, p);
+      w[mt][r] = (key < n && p != 0.0f) ? __fmul_rn(p, sm.vs[key]) : 0.0f;
+      wmax = fmaxf(wmax, w[mt][r]);
+    }
+  }
+  lsum = __fadd_rn(lsum, __shfl_xor_sync(0xffffffffu, lsum, 4));
+  lsum = __fadd_rn(lsum, __shfl_xor_sync(0xffffffffu, lsum, 8));
+  lsum = __fadd_rn(lsum, __shfl_xor_sync(0xffffffffu, lsum, 16));
+  wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, 4));
+  wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, 8));
+  wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, 16));
+  if (g == 0) {
+    sm.red_l[warp][c] = lsum;
+    sm.red_w[warp][c] = wmax;
+  }
+  __syncthreads();
+  // per-(split, head) exponent E: max_j w_j 2^E in [2^14, 2^15)
+  int E = 0;
+  {
+    const float wm = fmaxf(fmaxf(sm.red_w[0][c], sm.red_w[1][c]), fmaxf(sm.red_w[2][c], sm.red_w[3][c]));
+    if (wm > 0.0f) {
+      int ex;
+      frexpf(wm, &ex);
+      E = 15 - ex;
+      E = E < -120 ? -120 : (E > 120 ? 120 : E);
+    }
+  }
+  const float scaleE = inv::pow2f(E);
+  // packed (hi, lo) of w 2^E for keys g and g+8 of every m-tile
+  uint32_t pw_hi[4], pw_lo[4];
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    __half h0, l0, h1, l1;
+    inv::split_hi_lo(__fmul_rn(w[mt][0], scaleE), h0, l0);
+    inv::split_hi_lo(__fmul_rn(w[mt][1], scaleE), h1, l1);
+    pw_hi[mt] = pack_half2(h0, h1);
+    pw_lo[mt] = pack_half2(l0, l1);
+  }
+
+  if (lane == 0 && ok) ok = inv::mbar_wait(&sm.bar_v, 0, wait_ns, &sm.abort, status);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+
+  // --------------------------------------------------------------- values --
+  float o[8][4];
+#pragma unroll
+  for (int dt = 0; dt < 8; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.0f;
+  const int src1 = 4 * (2 * c) + (g >> 1), src2 = 4 * (2 * c + 1) + (g >> 1);
+  const bool want_lo = (g & 1) != 0;
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    const int kb = warp * 64 + mt * 16;
+    // B fragment of O^T = V^T W: rows k = keys, column g = head g/2 (hi/lo)
+    const uint32_t x1h = __shfl_sync(0xffffffffu, pw_hi[mt], src1);
+    const uint32_t x1l = __shfl_sync(0xffffffffu, pw_lo[mt], src1);
+    const uint32_t x2h = __shfl_sync(0xffffffffu, pw_hi[mt], src2);
+    const uint32_t x2l = __shfl_sync(0xffffffffu, pw_lo[mt], src2);
+    const uint32_t x1 = want_lo ? x1l : x1h, x2 = want_lo ? x2l : x2h;
+    const uint32_t b0 = __byte_perm(x1, x2, 0x5410);  // keys 2c, 2c+1
+    const uint32_t b1 = __byte_perm(x1, x2, 0x7632);  // keys 2c+8, 2c+9
+    if (ok && kb < n) {
+      const int lkey = kb + (lane >> 4) * 8 + (lane & 7);
+#pragma unroll
+      for (int dt = 0; dt < 8; ++dt) {
+        uint32_t a[4], ah[4], al[4];
+        ldsm_x4_t(code_addr(cbase, lkey, 16 * dt + ((lane >> 3) & 1) * 8), a);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) unpack_dual(a[i], ah[i], al[i]);
+        mma16816(o[dt], ah, b0, b1);
+        mma16816(o[dt], al, b0, b1);
+      }
+    }
+  }
+  // o[dt]: (d = 16dt + g, col 2c = w_hi head c), (d, col 2c+1 = w_lo), (d+8, ...)
+  __syncthreads();  // every warp is done reading V codes: reuse the buffer
+  float* xo = reinterpret_cast<float*>(sm.codes);  // [warp][head][128]
+  const float unscale = inv::pow2f(-E);
+#pragma unroll
+  for (int dt = 0; dt < 8; ++dt) {
+    const float v0 = __fmul_rn(__fmul_rn(__fadd_rn(o[dt][0], __fmul_rn(o[dt][1], 0x1p-11f)), 256.0f), unscale);
+    const float v1 = __fmul_rn(__fmul_rn(__fadd_rn(o[dt][2], __fmul_rn(o[dt][3], 0x1p-11f)), 256.0f), unscale);
+    xo[(warp * 4 + c) * 128 + 16 * dt + g] = v0;
+    xo[(warp * 4 + c) * 128 + 16 * dt + g + 8] = v1;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < 4 * 128; idx += THREADS) {
+    const int head = idx >> 7, d = idx & 127;
+    if (head >= G) continue;
+    float v = xo[(0 * 4 + head) * 128 + d];
+    v = __fadd_rn(v, xo[(1 * 4 + head) * 128 + d]);
+    v = __fadd_rn(v, xo[(2 * 4 + head) * 128 + d]);
+    v = __fadd_rn(v, xo[(3 * 4 + head) * 128 + d]);
+    part_o[(((int64_t)b * Hq + (int64_t)h * G + head) * S_max + s) * 128 + d] = v;
+  }
+  if (tid < G) {
+    const float Mh = fmaxf(fmaxf(sm.red_m[0][tid], sm.red_m[1][tid]), fmaxf(sm.red_m[2][tid], sm.red_m[3][tid]));
+    float l = sm.red_l[0][tid];
+    l = __fadd_rn(l, sm.red_l[1][tid]);
+    l = __fadd_rn(l, sm.red_l[2][tid]);
+    l = __fadd_rn(l, sm.red_l[3][tid]);
+    part_ml[((int64_t)b * Hq + (int64_t)h * G + tid) * S_max + s] = make_float2(Mh, l);
+  }
+  // No copy may still be landing in this CTA's shared memory when it exits
+  // (only possible after a timed-out wait; immediate otherwise).
+  if (tid == 0) {
+    inv::mbar_wait(&sm.bar_k, 0, wait_ns, nullptr, status);
+    if (v_issued) inv::mbar_wait(&sm.bar_v, 0, wait_ns, nullptr, status);
+  }
+}
+
+// One warp per (row, head): fold splits s = 0, 1, ... in order.
+__global__ void attn_combine_kernel(const float* __restrict__ part_o, const float2* __restrict__ part_ml,
+                                    const int32_t* __restrict__ len, int B, int Hq, int S_max, int len_limit,
+                                    float* __restrict__ out, __half* __restrict__ out_hi, __half* __restrict__ out_lo,
+                                    int* status) {
+  const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= (int64_t)B * Hq) return;
+  const int b = (int)(wid / Hq);
+  const int L = len[b];
+  float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (L >= 1 && L <= len_limit) {
+    const int S = (L + SPLIT - 1) / SPLIT;
+    const float2* ml = part_ml + wid * S_max;
+    float M = -INFINITY;
+    for (int s = 0; s < S; ++s) M = fmaxf(M, ml[s].x);
+    float l = 0.0f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < S; ++s) {
+      const float2 v = ml[s];
+      const float f = expf(__fsub_rn(v.x, M));
+      l = __fadd_rn(l, __fmul_rn(v.y, f));
+      const float4 po = reinterpret_cast<const float4*>(part_o + (wid * S_max + s) * 128)[lane];
+      acc.x = __fadd_rn(acc.x, __fmul_rn(po.x, f));
+      acc.y = __fadd_rn(acc.y, __fmul_rn(po.y, f));
+      acc.z = __fadd_rn(acc.z, __fmul_rn(po.z, f));
+      acc.w = __fadd_rn(acc.w, __fmul_rn(po.w, f));
+    }
+    res = make_float4(__fdiv_rn(acc.x, l), __fdiv_rn(acc.y, l), __fdiv_rn(acc.z, l), __fdiv_rn(acc.w, l));
+  }
+  reinterpret_cast<float4*>(out + wid * 128)[lane] = res;
+  if (out_hi) {
+    __half h[4], lo[4];
+    inv::split_hi_lo(res.x, h[0], lo[0]);
+    inv::split_hi_lo(res.y, h[1], lo[1]);
+    inv::split_hi_lo(res.z, h[2], lo[2]);
+    inv::split_hi_lo(res.w, h[3], lo[3]);
+    if (inv::f16_overflow(res.x) | inv::f16_overflow(res.y) | inv::f16_overflow(res.z) | inv::f16_overflow(res.w))
+      record_status(status, INV_ERR_RANGE);
+    uint2 hv, lv;
+    hv.x = pack_half2(h[0], h[1]);
+    hv.y = pack_half2(h[2], h[3]);
+    lv.x = pack_half2(lo[0], lo[1]);
+    lv.y = pack_half2(lo[2], lo[3]);
+    reinterpret_cast<uint2*>(out_hi + wid * 128)[lane] = hv;
+    reinterpret_cast<uint2*>(out_lo + wid * 128)[lane] = lv;
+  }
+}
+
+bool g_attn_attr[64] = {};
+
+}  // namespace
+
+namespace inv {
+
+static int splits_for(int max_len_bound) { return (max_len_bound + SPLIT - 1) / SPLIT; }
+
+size_t attn_workspace_bytes(int B, int Hq, int max_len_bound) {
+  const size_t S = (size_t)splits_for(max_len_bound);
+  return (size_t)B * Hq * S * (128 * sizeof(float) + sizeof(float2));
+}
+
+int launch_attention(const float* q, int B, int Hq, const inv_kv_cache& c, const int32_t* slot, const int32_t* len,
+                     int max_len_bound, float sigma, float* out, uint16_t* out_hi, uint16_t* out_lo, void* ws,
+                     cudaStream_t s) {
+  if (B == 0) return INV_OK;
+  const int S_max = splits_for(max_len_bound);
+  float* part_o = static_cast<float*>(ws);
+  float2* part_ml = reinterpret_cast<float2*>(part_o + (size_t)B * Hq * S_max * 128);
+  const uint64_t rows = (uint64_t)c.n_slots * c.n_kv_heads * c.max_len;
+  CUtensorMap tk, tv;
+  int rc = make_tensor_map_2d(&tk, c.k, CU_TENSOR_MAP_DATA_TYPE_UINT16, 128, rows, 256, 64, 64,
+                              CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != INV_OK) return rc;
+  rc = make_tensor_map_2d(&tv, c.v, CU_TENSOR_MAP_DATA_TYPE_UINT16, 128, rows, 256, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != INV_OK) return rc;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !g_attn_attr[dev]) {
+    if (cudaFuncSetAttribute(attn_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem) !=
+        cudaSuccess)
+      return INV_ERR_CUDA;
+    g_attn_attr[dev] = true;
+  }
+  dim3 grid(S_max, c.n_kv_heads, B);
+  attn_split_kernel<<<grid, THREADS, kAttnSmem, s>>>(tk, tv, q, c.k_scale, c.v_scale, slot, len, Hq, c.n_kv_heads,
+                                                     c.n_slots, c.max_len, max_len_bound, S_max, sigma, part_o, part_ml,
+                                                     status_ptr(), wait_limit_ns());
+  INV_CHECK_LAUNCH();
+  const int64_t warps = (int64_t)B * Hq;
+  attn_combine_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(
+      part_o, part_ml, len, B, Hq, S_max, max_len_bound, out, reinterpret_cast<__half*>(out_hi),
+      reinterpret_cast<__half*>(out_lo), status_ptr());
+  INV_CHECK_LAUNCH();
+  return INV_OK;
+}
+
+}  // namespace inv
+
+extern "C" {
+
+size_t attn_decode_workspace_size(int B, int n_heads, int max_len_bound) {
+  if (B <= 0 || n_heads <= 0 || max_len_bound <= 0) return 0;
+  return inv::attn_workspace_bytes(B, n_heads, max_len_bound);
+}
+
+int attn_decode_fixedsplit(const float* q, int B, int n_heads, const inv_kv_cache* cache, const int32_t* slot,
+                           const int32_t* len, int max_len_bound, int split, float softmax_scale, float* out,
+                           uint16_t* out_hi, uint16_t* out_lo, void* workspace, size_t ws_bytes, inv_stream stream) {
+  if (!cache || B < 0 || n_heads <= 0) return INV_ERR_INVALID_ARG;
+  if (split != INV_KV_SPLIT) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (cache->head_dim != INV_HEAD_DIM || cache->n_kv_heads <= 0 || n_heads % cache->n_kv_heads != 0)
+    return INV_ERR_UNSUPPORTED_SHAPE;
+  const int G = n_heads / cache->n_kv_heads;
+  if (G != 1 && G != 2 && G != 4) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (cache->max_len <= 0 || cache->max_len % 64 != 0 || cache->n_slots <= 0) return INV_ERR_INVALID_ARG;
+  if ((uint64_t)cache->n_slots * cache->n_kv_heads * cache->max_len >= (1ull << 31)) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0) return INV_OK;
+  if (B > 65535) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (!q || !slot || !len || !out || !cache->k || !cache->v || !cache->k_scale || !cache->v_scale || !workspace)
+    return INV_ERR_INVALID_ARG;
+  if ((out_hi == nullptr) != (out_lo == nullptr)) return INV_ERR_INVALID_ARG;
+  if (!inv::aligned16(cache->k) || !inv::aligned16(cache->v) || !inv::aligned16(out) || !inv::aligned16(workspace))
+    return INV_ERR_INVALID_ARG;
+  if (out_hi && ((reinterpret_cast<uintptr_t>(out_hi) | reinterpret_cast<uintptr_t>(out_lo)) & 7u))
+    return INV_ERR_INVALID_ARG;
+  const int mlb = max_len_bound > 0 ? (max_len_bound < cache->max_len ? max_len_bound : cache->max_len) : cache->max_len;
+  if (ws_bytes < inv::attn_workspace_bytes(B, n_heads, mlb)) return INV_ERR_WORKSPACE;
+  return inv::launch_attention(q, B, n_heads, *cache, slot, len, mlb, softmax_scale, out, out_hi, out_lo, workspace,
+                               static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,283 @@
+// Error-compensated GEMM on 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// HEAL explainer, section "2. 「誤差補償」のトリック（計算用）": a main product in
+// 16-bit containers plus a clean-up product that catches what it spilled.
+// With a = a_hi + 2^-11 a_lo and w 2^e = w_hi + 2^-11 w_lo (binary16 pairs):
+//   y = ( sum a_hi w_hi  +  2^-11 sum (a_hi w_lo + a_lo w_hi) ) 2^-e   [+ residual]
+// Batch invariance ("Defeating Nondeterminism" summary, table row MatMul):
+// ONE tile (128 x 64), ONE K order, no split-K, whatever M is.
+//
+// Per 128 x 64 output tile and per 64-wide K block, the MMA thread issues for
+// each 16-wide K step:
+//   MMA1  D[0:128)  (+)= A_hi * [W_hi ; W_lo]^T   (N = 128: columns 0..63 "hh",
+//                                                  64..127 the first cross term)
+//   MMA2  D[64:128) += A_lo * W_hi^T              (N = 64: second cross term)
+// Accumulation runs in tensor memory over a group of 256 K values (4 blocks),
+// then the epilogue warps read the group (tcgen05.ld) and add it to fp32
+// registers with round-to-nearest adds, groups in ascending K.  Restarting
+// the tensor-memory accumulator every 256 K bounds the error of the tensor
+// core's internal accumulation, whatever K is.  Two group buffers (2 x 128
+// TMEM columns) let the MMAs of group g+1 overlap the drain of group g.
+//
+// Warp roles (320 threads): warp 0 = TMA producer, warp 1 = TMEM allocator +
+// MMA issuer, warps 2..9 = epilogue (warp w reads TMEM lanes 32*(w%4).., the
+// column half (w-2)/4).  Persistent grid over tiles ordered N-panel-major so a
+// wave of CTAs shares weight panels and the A rows stay in L2.
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+constexpr int BM = INV_GEMM_BM;            // 128
+constexpr int BN = INV_GEMM_BN;            // 64
+constexpr int BK = INV_GEMM_BK;            // 64
+constexpr int STAGES = 4;
+constexpr int GROUP_KB = INV_GEMM_KGROUP / BK;  // 4
+constexpr int A_BYTES = BM * BK * 2;       // 16 KB
+constexpr int W_BYTES = 2 * BN * BK * 2;   // 16 KB: 64 hi rows then 64 lo rows
+constexpr int STAGE_BYTES = 2 * A_BYTES + W_BYTES;
+constexpr int ACC_COLS = 2 * BN;           // hh | cross
+constexpr int TMEM_COLS = 2 * ACC_COLS;    // two group buffers
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
+constexpr uint32_t IDESC_N128 = inv::idesc_f16_f32(128, 128);
+constexpr uint32_t IDESC_N64 = inv::idesc_f16_f32(128, 64);
+
+struct __align__(1024) GemmSmem {
+  uint8_t stage[STAGES][STAGE_BYTES];
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t kSmemBytes = sizeof(GemmSmem) + 1024;
+
+__global__ void __launch_bounds__(THREADS, 1)
+    comp_gemm_kernel(const __grid_constant__ CUtensorMap tm_ahi, const __grid_constant__ CUtensorMap tm_alo,
+                     const __grid_constant__ CUtensorMap tm_w, const int8_t* __restrict__ col_exp, float* y,
+                     int64_t ld_y, const float* residual, int64_t ld_r, int M, int N, int K, int* status,
+                     long long wait_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_m = (M + BM - 1) / BM;
+  const int n_tiles = tiles_m * (N / BN);
+  const int nkb = K / BK;
+  const int ngroups = (nkb + GROUP_KB - 1) / GROUP_KB;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      inv::mbar_init(&sm.full[s], 1);
+      inv::mbar_init(&sm.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      inv::mbar_init(&sm.tfull[b], 1);
+      inv::mbar_init(&sm.tempty[b], EPI_WARPS);
+    }
+    inv::mbar_init(&sm.done, 1);
+    sm.abort = 0;
+    inv::fence_mbar_init();
+  }
+  if (warp == 1) {
+    inv::tmem_alloc(&sm.tmem_base, TMEM_COLS);
+    inv::tmem_relinquish();
+  }
+  inv::tc_fence_before();
+  __syncthreads();
+  inv::tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t issued_mask = 0, last_phase_mask = 0;
+      for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        const int nt = tile / tiles_m, mt = tile - nt * tiles_m;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!inv::mbar_wait(&sm.empty[stage], phase ^ 1u, wait_ns, abort_flag, status)) goto producer_done;
+          uint8_t* st = sm.stage[stage];
+          inv::mbar_arrive_expect_tx(&sm.full[stage], STAGE_BYTES);
+          inv::tma_load_2d(st, &tm_ahi, &sm.full[stage], kb * BK, mt * BM);
+          inv::tma_load_2d(st + A_BYTES, &tm_alo, &sm.full[stage], kb * BK, mt * BM);
+          inv::tma_load_2d(st + 2 * A_BYTES, &tm_w, &sm.full[stage], kb * BK, nt * 2 * BN);
+          issued_mask |= 1u << stage;
+          last_phase_mask = (last_phase_mask & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    producer_done:
+      // Every load issued must have landed before the CTA may exit.
+      for (int s = 0; s < STAGES; ++s)
+        if (issued_mask & (1u << s))
+          inv::mbar_wait(&sm.full[s], (last_phase_mask >> s) & 1u, wait_ns, nullptr, status);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, g = 0;
+      for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        for (int grp = 0; grp < ngroups; ++grp, ++g) {
+          const uint32_t buf = g & 1u, tph = (g >> 1) & 1u;
+          if (!inv::mbar_wait(&sm.tempty[buf], tph ^ 1u, wait_ns, abort_flag, status)) goto mma_done;
+          inv::tc_fence_after();
+          const uint32_t d = tmem + buf * ACC_COLS;
+          const int kb0 = grp * GROUP_KB;
+          const int kb1 = min(nkb, kb0 + GROUP_KB);
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!inv::mbar_wait(&sm.full[stage], phase, wait_ns, abort_flag, status)) goto mma_done;
+            inv::tc_fence_after();
+            const uint32_t base = inv::smem_u32(sm.stage[stage]);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ahi = inv::sw128_kmajor_desc(base + kk * 32);
+              const uint64_t alo = inv::sw128_kmajor_desc(base + A_BYTES + kk * 32);
+              const uint64_t bw = inv::sw128_kmajor_desc(base + 2 * A_BYTES + kk * 32);
+              inv::umma_f16(d, ahi, bw, IDESC_N128, (kb > kb0 || kk > 0) ? 1u : 0u);
+              inv::umma_f16(d + BN, alo, bw, IDESC_N64, 1u);
+            }
+            inv::umma_commit(&sm.empty[stage]);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          inv::umma_commit(&sm.tfull[buf]);
+        }
+      }
+    mma_done:
+      // Every MMA issued must have completed before TMEM is released.
+      inv::umma_commit(&sm.done);
+      inv::mbar_wait(&sm.done, 0, wait_ns, nullptr, status);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue --
+    const int quarter = warp & 3;          // TMEM lanes 32*quarter .. +31
+    const int half = (warp - 2) >> 2;      // output columns 32*half .. +31
+    uint32_t g = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+      const int nt = tile / tiles_m, mt = tile - nt * tiles_m;
+      float acc_h[32], acc_x[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) acc_h[i] = acc_x[i] = 0.0f;
+      for (int grp = 0; grp < ngroups; ++grp, ++g) {
+        const uint32_t buf = g & 1u, tph = (g >> 1) & 1u;
+        int okw = 1;
+        if (lane == 0) okw = inv::mbar_wait(&sm.tfull[buf], tph, wait_ns, abort_flag, status) ? 1 : 0;
+        okw = __shfl_sync(0xffffffffu, okw, 0);  // keep the warp converged for tcgen05.ld
+        if (!okw) goto epi_done;
+        inv::tc_fence_after();
+        const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * ACC_COLS + half * 32;
+        uint32_t rh[32], rx[32];
+        inv::tmem_ld_32x32(ta, rh);
+        inv::tmem_ld_32x32(ta + BN, rx);
+        inv::tmem_wait_ld();
+        inv::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) inv::mbar_arrive(&sm.tempty[buf]);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          acc_h[i] = __fadd_rn(acc_h[i], __uint_as_float(rh[i]));
+          acc_x[i] = __fadd_rn(acc_x[i], __uint_as_float(rx[i]));
+        }
+      }
+      {
+        const int row = mt * BM + quarter * 32 + lane;
+        if (row < M) {
+          const int col0 = nt * BN + half * 32;
+          float* yr = y + (int64_t)row * ld_y + col0;
+          const float* rr = residual ? residual + (int64_t)row * ld_r + col0 : nullptr;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const char4 e4 = *reinterpret_cast<const char4*>(col_exp + col0 + i);
+            const int ev[4] = {e4.x, e4.y, e4.z, e4.w};
+            float o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float t = __fadd_rn(acc_h[i + j], __fmul_rn(acc_x[i + j], 0x1p-11f));
+              o[j] = __fmul_rn(t, inv::pow2f(-ev[j]));
+            }
+            if (rr) {
+              const float4 r4 = *reinterpret_cast<const float4*>(rr + i);
+              o[0] = __fadd_rn(o[0], r4.x);
+              o[1] = __fadd_rn(o[1], r4.y);
+              o[2] = __fadd_rn(o[2], r4.z);
+              o[3] = __fadd_rn(o[3], r4.w);
+            }
+            *reinterpret_cast<float4*>(yr + i) = make_float4(o[0], o[1], o[2], o[3]);
+          }
+        }
+      }
+    }
+  epi_done:;
+  }
+
+  inv::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    inv::tc_fence_after();
+    inv::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+bool g_attr_set[64] = {};
+
+}  // namespace
+
+namespace inv {
+
+int launch_comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
+                     const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
+                     const float* residual, int64_t ld_r, cudaStream_t s) {
+  if (M == 0) return INV_OK;
+  CUtensorMap ta, tl, tw;
+  int rc = make_tensor_map_2d(&ta, a_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)M,
+                              (uint64_t)ld_a * 2, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != INV_OK) return rc;
+  rc = make_tensor_map_2d(&tl, a_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)M, (uint64_t)ld_a * 2,
+                          BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != INV_OK) return rc;
+  rc = make_tensor_map_2d(&tw, w_packed, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)N * 2,
+                          (uint64_t)K * 2, BK, 2 * BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != INV_OK) return rc;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !g_attr_set[dev]) {
+    if (cudaFuncSetAttribute(comp_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
+        cudaSuccess)
+      return INV_ERR_CUDA;
+    g_attr_set[dev] = true;
+  }
+  const int64_t tiles = ((M + BM - 1) / BM) * (N / BN);
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  comp_gemm_kernel<<<grid, THREADS, kSmemBytes, s>>>(ta, tl, tw, col_exp, y, ld_y, residual, ld_r, (int)M, N, K,
+                                                     status_ptr(), wait_limit_ns());
+  INV_CHECK_LAUNCH();
+  return INV_OK;
+}
+
+}  // namespace inv
+
+extern "C" int comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
+                         const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
+                         const float* residual, int64_t ld_r, inv_stream stream) {
+  if (M < 0 || K <= 0 || N <= 0) return INV_ERR_INVALID_ARG;
+  if (K % BK != 0 || N % BN != 0) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return INV_OK;
+  if (M > 0x7fffffffLL) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (!a_hi || !a_lo || !w_packed || !col_exp || !y) return INV_ERR_INVALID_ARG;
+  if (ld_a < K || ld_a % 8 != 0 || ld_y < N || ld_y % 4 != 0) return INV_ERR_INVALID_ARG;
+  if (!inv::aligned16(a_hi) || !inv::aligned16(a_lo) || !inv::aligned16(w_packed) || !inv::aligned16(y))
+    return INV_ERR_INVALID_ARG;
+  if (residual && (ld_r < N || ld_r % 4 != 0 || !inv::aligned16(residual))) return INV_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(col_exp) & 3u) != 0) return INV_ERR_INVALID_ARG;
+  return inv::launch_comp_gemm(a_hi, a_lo, M, K, ld_a, w_packed, col_exp, N, y, ld_y, residual, ld_r,
+                               static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,142 @@
+// decode_layer: one LLaMA-style block over B token rows, composed from the
+// library's kernels and nothing else (stream-ordered, no host synchronisation).
+//
+// HEAL explainer, section "真の犯人（「カーネル境界」）": precision is lost at kernel
+// boundaries when intermediates are stored in smaller containers.  Here every
+// tensor crossing a kernel boundary is either fp32 or an exact binary16 hi/lo
+// pair; the only lossy store is the INT16 KV cache the method prescribes.
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct LayerWs {
+  uint16_t *h_hi, *h_lo;
+  float* qkv;
+  float* q_rot;
+  int32_t* lens;
+  void* attn;
+  float* o;
+  uint16_t *o_hi, *o_lo;
+  float* x1;
+  uint16_t *h2_hi, *h2_lo;
+  float* gu;
+  uint16_t *a_hi, *a_lo;
+  size_t bytes;
+};
+
+LayerWs carve(const inv_layer_config& c, int B, int mlb, uint8_t* base) {
+  LayerWs w{};
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    uint8_t* p = base ? base + off : nullptr;
+    off += align256(n);
+    return p;
+  };
+  const size_t H = c.hidden, F = c.ffn, QD = (size_t)c.n_heads * 128;
+  const size_t NQKV = (size_t)(c.n_heads + 2 * c.n_kv_heads) * 128;
+  w.h_hi = reinterpret_cast<uint16_t*>(take(B * H * 2));
+  w.h_lo = reinterpret_cast<uint16_t*>(take(B * H * 2));
+  w.qkv = reinterpret_cast<float*>(take(B * NQKV * 4));
+  w.q_rot = reinterpret_cast<float*>(take(B * QD * 4));
+  w.lens = reinterpret_cast<int32_t*>(take(B * 4));
+  w.attn = take(inv::attn_workspace_bytes(B, c.n_heads, mlb));
+  w.o = reinterpret_cast<float*>(take(B * QD * 4));
+  w.o_hi = reinterpret_cast<uint16_t*>(take(B * QD * 2));
+  w.o_lo = reinterpret_cast<uint16_t*>(take(B * QD * 2));
+  w.x1 = reinterpret_cast<float*>(take(B * H * 4));
+  w.h2_hi = reinterpret_cast<uint16_t*>(take(B * H * 2));
+  w.h2_lo = reinterpret_cast<uint16_t*>(take(B * H * 2));
+  w.gu = reinterpret_cast<float*>(take(B * 2 * F * 4));
+  w.a_hi = reinterpret_cast<uint16_t*>(take(B * F * 2));
+  w.a_lo = reinterpret_cast<uint16_t*>(take(B * F * 2));
+  w.bytes = off;
+  return w;
+}
+
+int validate(const inv_layer_config* cfg, const inv_kv_cache* cache) {
+  if (!cfg || !cache) return INV_ERR_INVALID_ARG;
+  if (cfg->head_dim != INV_HEAD_DIM || cache->head_dim != INV_HEAD_DIM) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (cfg->hidden <= 0 || cfg->ffn <= 0 || cfg->n_heads <= 0 || cfg->n_kv_heads <= 0 || cfg->max_pos <= 0)
+    return INV_ERR_INVALID_ARG;
+  if (cfg->hidden % 64 != 0 || cfg->ffn % 64 != 0) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (cfg->n_heads % cfg->n_kv_heads != 0) return INV_ERR_UNSUPPORTED_SHAPE;
+  const int G = cfg->n_heads / cfg->n_kv_heads;
+  if (G != 1 && G != 2 && G != 4) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (cache->n_kv_heads != cfg->n_kv_heads || cache->max_len <= 0 || cache->max_len % 64 != 0 ||
+      cache->n_slots <= 0)
+    return INV_ERR_INVALID_ARG;
+  if ((uint64_t)cache->n_slots * cache->n_kv_heads * cache->max_len >= (1ull << 31)) return INV_ERR_UNSUPPORTED_SHAPE;
+  return INV_OK;
+}
+
+int bound_of(const inv_kv_cache* cache, int max_len_bound) {
+  return max_len_bound > 0 ? (max_len_bound < cache->max_len ? max_len_bound : cache->max_len) : cache->max_len;
+}
+
+#define INV_TRY(expr)          \
+  do {                         \
+    const int rc_ = (expr);    \
+    if (rc_ != INV_OK) return rc_; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+size_t decode_layer_workspace_size(const inv_layer_config* cfg, int B, int max_len_bound) {
+  if (!cfg || B <= 0 || cfg->hidden <= 0 || cfg->ffn <= 0 || cfg->n_heads <= 0 || cfg->n_kv_heads <= 0) return 0;
+  const int mlb = max_len_bound > 0 ? max_len_bound : 1;
+  return carve(*cfg, B, mlb, nullptr).bytes;
+}
+
+int decode_layer(const inv_layer_config* cfg, const inv_layer_weights* w, const inv_kv_cache* cache,
+                 const float* x_in, const int32_t* slot, const int32_t* pos, int B, int max_len_bound, float* x_out,
+                 void* workspace, size_t ws_bytes, inv_stream stream) {
+  INV_TRY(validate(cfg, cache));
+  if (!w || B < 0) return INV_ERR_INVALID_ARG;
+  if (B == 0) return INV_OK;
+  if (B > 65535) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (!x_in || !x_out || !slot || !pos || !workspace || x_in == x_out) return INV_ERR_INVALID_ARG;
+  if (!w->w_qkv || !w->e_qkv || !w->w_o || !w->e_o || !w->w_gu || !w->e_gu || !w->w_down || !w->e_down ||
+      !w->g_attn || !w->g_mlp || !w->rope_cos || !w->rope_sin)
+    return INV_ERR_INVALID_ARG;
+  if (!cache->k || !cache->v || !cache->k_scale || !cache->v_scale) return INV_ERR_INVALID_ARG;
+  if (!inv::aligned16(x_in) || !inv::aligned16(x_out) || !inv::aligned16(workspace) || !inv::aligned16(w->rope_cos) ||
+      !inv::aligned16(w->rope_sin) || !inv::aligned16(w->g_attn) || !inv::aligned16(w->g_mlp) ||
+      !inv::aligned16(cache->k) || !inv::aligned16(cache->v))
+    return INV_ERR_INVALID_ARG;
+  const int mlb = bound_of(cache, max_len_bound);
+  const LayerWs ws = carve(*cfg, B, mlb, static_cast<uint8_t*>(workspace));
+  if (ws_bytes < ws.bytes) return INV_ERR_WORKSPACE;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int H = cfg->hidden, F = cfg->ffn, Hq = cfg->n_heads, Hkv = cfg->n_kv_heads;
+  const int QD = Hq * 128, NQKV = (Hq + 2 * Hkv) * 128;
+
+  // 1. h = rmsnorm(x) -> hi/lo
+  INV_TRY(inv::launch_rmsnorm(x_in, w->g_attn, B, H, cfg->eps, nullptr, ws.h_hi, ws.h_lo, s));
+  // 2. qkv = h W_qkv
+  INV_TRY(inv::launch_comp_gemm(ws.h_hi, ws.h_lo, B, H, H, w->w_qkv, w->e_qkv, NQKV, ws.qkv, NQKV, nullptr, 0, s));
+  // 3. rotary embedding of q and k; k, v -> INT16 cache; len = pos + 1
+  INV_TRY(inv::launch_rope_quant(ws.qkv, B, Hq, *cache, slot, pos, w->rope_cos, w->rope_sin, cfg->max_pos, ws.q_rot,
+                                 ws.lens, s));
+  // 4-5. fixed-split attention + ordered combine -> o hi/lo
+  INV_TRY(inv::launch_attention(ws.q_rot, B, Hq, *cache, slot, ws.lens, mlb, cfg->softmax_scale, ws.o, ws.o_hi,
+                                ws.o_lo, ws.attn, s));
+  // 6. x1 = x + o W_o
+  INV_TRY(inv::launch_comp_gemm(ws.o_hi, ws.o_lo, B, QD, QD, w->w_o, w->e_o, H, ws.x1, H, x_in, H, s));
+  // 7. h2 = rmsnorm(x1) -> hi/lo
+  INV_TRY(inv::launch_rmsnorm(ws.x1, w->g_mlp, B, H, cfg->eps, nullptr, ws.h2_hi, ws.h2_lo, s));
+  // 8. [gate | up] = h2 W_gu
+  INV_TRY(inv::launch_comp_gemm(ws.h2_hi, ws.h2_lo, B, H, H, w->w_gu, w->e_gu, 2 * F, ws.gu, 2 * F, nullptr, 0, s));
+  // 9. a = silu(gate) * up -> hi/lo
+  INV_TRY(inv::launch_swiglu_split(ws.gu, B, F, ws.a_hi, ws.a_lo, s));
+  // 10. out = x1 + a W_down
+  INV_TRY(inv::launch_comp_gemm(ws.a_hi, ws.a_lo, B, F, F, w->w_down, w->e_down, H, x_out, H, ws.x1, H, s));
+  return INV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,32 @@
+// Internal launchers shared between translation units (no validation: the
+// public entry points and decode_layer validate before calling these).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "invnum.h"
+
+namespace inv {
+
+int launch_rmsnorm(const float* x, const float* gamma, int64_t rows, int hidden, float eps, float* y,
+                   uint16_t* yh, uint16_t* yl, cudaStream_t s);
+
+int launch_rope_quant(const float* qkv, int T, int Hq, const inv_kv_cache& c, const int32_t* slot,
+                      const int32_t* pos, const float* rope_cos, const float* rope_sin, int max_pos, float* q_out,
+                      int32_t* len_out, cudaStream_t s);
+
+int launch_swiglu_split(const float* gu, int64_t T, int F, uint16_t* ah, uint16_t* al, cudaStream_t s);
+
+int launch_comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
+                     const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
+                     const float* residual, int64_t ld_r, cudaStream_t s);
+
+// Workspace layout of the attention: partial (m, l) and partial o per
+// (row, head, split).
+size_t attn_workspace_bytes(int B, int Hq, int max_len_bound);
+int launch_attention(const float* q, int B, int Hq, const inv_kv_cache& c, const int32_t* slot, const int32_t* len,
+                     int max_len_bound, float sigma, float* out, uint16_t* out_hi, uint16_t* out_lo, void* ws,
+                     cudaStream_t s);
+
+}  // namespace inv

@@ -1,0 +1,103 @@
+"""The full decode layer on the GPU: parity with the oracle layer, bit-identity
+across batch size / composition, and chunked versus one-shot prefill."""
+import numpy as np
+import pytest
+import torch
+
+from invariant_numerics_b200 import synth
+from oracle import reference as ref
+
+from gpu_helpers import TOL, dev, host, rowwise_err, status
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def inv():
+    from invariant_numerics_b200 import invnum
+    assert invnum.inv_get_device_status() == invnum.INV_OK
+    return invnum
+
+
+def make_layer(inv, H, Hq, Hkv, F, max_pos, seed=0):
+    D = 128
+    s = lambda i, shape: synth.normal(shape, seed=seed, stream=i, std=0.02)
+    p = ref.LayerParams(wq=s(1, (H, Hq * D)), wk=s(2, (H, Hkv * D)), wv=s(3, (H, Hkv * D)), wo=s(4, (Hq * D, H)),
+                        w_gate=s(5, (H, F)), w_up=s(6, (H, F)), w_down=s(7, (F, H)),
+                        g_attn=synth.uniform(H, seed=seed, stream=8, lo=0.5, hi=1.5),
+                        g_mlp=synth.uniform(H, seed=seed, stream=9, lo=0.5, hi=1.5),
+                        n_heads=Hq, n_kv_heads=Hkv, head_dim=D)
+    cfg = inv.LayerConfig(hidden=H, n_heads=Hq, n_kv_heads=Hkv, ffn=F, max_pos=max_pos)
+    w = inv.LayerWeights(cfg, dev(p.wq), dev(p.wk), dev(p.wv), dev(p.wo), dev(p.w_gate), dev(p.w_up),
+                         dev(p.w_down), dev(p.g_attn), dev(p.g_mlp))
+    return p, cfg, w
+
+
+SMALL = dict(H=256, Hq=8, Hkv=2, F=512, max_pos=1024)
+
+
+def test_layer_parity_small(inv):
+    p, cfg, w = make_layer(inv, **SMALL)
+    n_slots, max_len = 3, 512
+    oc = ref.KVCache.empty(n_slots, 2, max_len, 128)
+    gc = inv.KVCache(n_slots=n_slots, n_kv_heads=2, max_len=max_len)
+    # prefill three sequences of different lengths in chunks, then decode
+    steps = [
+        (np.zeros(300, np.int32), np.arange(300, dtype=np.int32)),
+        (np.ones(37, np.int32), np.arange(37, dtype=np.int32)),
+        (np.full(5, 2, np.int32), np.arange(5, dtype=np.int32)),
+        (np.array([0, 1, 2], np.int32), np.array([300, 37, 5], np.int32)),
+        (np.array([2, 0], np.int32), np.array([6, 301], np.int32)),
+    ]
+    for i, (slot, pos) in enumerate(steps):
+        x = synth.normal((len(slot), SMALL["H"]), seed=100 + i)
+        y = inv.decode_layer(cfg, w, gc, dev(x), dev(slot), dev(pos))
+        want = ref.decode_layer(p, oc, x, slot, pos)
+        err = rowwise_err(host(y), want)
+        assert err.max() <= TOL, (i, err.max())
+    assert status() == inv.INV_OK
+
+
+def test_layer_batch_invariance_and_composition(inv):
+    p, cfg, w = make_layer(inv, **SMALL, seed=1)
+    n_seq, ctx = 128, 200
+    gc = inv.KVCache(n_slots=n_seq, n_kv_heads=2, max_len=256)
+    # fill every slot with a 200-token context
+    for b in range(0, n_seq, 16):
+        slots = np.repeat(np.arange(b, b + 16, dtype=np.int32), ctx)
+        pos = np.tile(np.arange(ctx, dtype=np.int32), 16)
+        x = synth.normal((len(slots), SMALL["H"]), seed=7, stream=b)
+        inv.decode_layer(cfg, w, gc, dev(x), dev(slots), dev(pos))
+    x = synth.normal((n_seq, SMALL["H"]), seed=8)
+    pos = np.full(n_seq, ctx, np.int32)
+    ref_out = None
+    for B in (128, 32, 8, 1):
+        perm = synth.permutation(n_seq, seed=B)
+        outs = np.zeros((n_seq, SMALL["H"]), np.float32)
+        for a in range(0, n_seq, B):
+            idx = perm[a:a + B]
+            y = inv.decode_layer(cfg, w, gc, dev(x[idx]), dev(idx.astype(np.int32)), dev(pos[idx]))
+            outs[idx] = host(y)
+        if ref_out is None:
+            ref_out = outs
+        else:
+            assert np.array_equal(outs.view(np.int32), ref_out.view(np.int32)), B
+    assert status() == inv.INV_OK
+
+
+def test_chunked_prefill_matches_one_shot(inv):
+    p, cfg, w = make_layer(inv, **SMALL, seed=2)
+    T = 600
+    x = synth.normal((T, SMALL["H"]), seed=9)
+    pos = np.arange(T, dtype=np.int32)
+    a = inv.KVCache(n_slots=1, n_kv_heads=2, max_len=1024)
+    b = inv.KVCache(n_slots=1, n_kv_heads=2, max_len=1024)
+    one = inv.decode_layer(cfg, w, a, dev(x), dev(np.zeros(T, np.int32)), dev(pos))
+    parts = []
+    for lo, hi in ((0, 256), (256, 257), (257, 512), (512, 600)):
+        parts.append(inv.decode_layer(cfg, w, b, dev(x[lo:hi].copy()), dev(np.zeros(hi - lo, np.int32)),
+                                      dev(pos[lo:hi].copy())))
+    chunked = torch.cat(parts)
+    assert torch.equal(one.view(torch.int32), chunked.view(torch.int32))
+    assert torch.equal(a.k, b.k) and torch.equal(a.v, b.v)
+    assert torch.equal(a.k_scale, b.k_scale) and torch.equal(a.v_scale, b.v_scale)
