@@ -1,0 +1,529 @@
+#!/usr/bin/env python
+"""Benchmark of the batch-invariant, error-compensated decode layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (one step): one decode_layer call -- RMSNorm, compensated QKV GEMM,
+rotary embedding + INT16 quantisation into the cache, fixed-split attention
+over a 2048-token INT16 KV cache, compensated output GEMM + residual,
+RMSNorm, compensated gate/up GEMM, SwiGLU, compensated down GEMM + residual --
+for B = 128 sequences of a 7B-like layer (hidden 4096, 32 query / 8 KV heads
+of 128, MLP 11008).  Weights are random N(0, 0.02) fp32 packed once into the
+hi/lo binary16 image; the KV cache holds 2047 synthetic tokens per sequence
+and every step decodes position 2047 (2048 keys).  The rows come in a seeded
+shuffled order of the cache slots.
+
+Reported: tokens/s of the whole job (value), the device-resident step time,
+an end-to-end figure through the C ABI with host buffers (H2D of the step's
+inputs and D2H of its output inside the timed region), per-kernel times from
+CUDA events recorded around every kernel inside the timed region, the
+roofline of the dominant kernel, SM clocks sampled during the run, and the
+CPU oracle timed on a bounded sample of the same workload.  Components: the
+compensated GEMM at the GEMM-sweep shapes and the decode attention at the
+ragged-length shape, each against its roofline.
+
+Multi-GPU: replicas only -- every rank runs the full per-GPU workload on its
+own device (weak scaling); the only cross-rank traffic is a barrier and the
+max of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+H, HQ, HKV, D, F = 4096, 32, 8, 128, 11008
+BATCH, KV_LEN = 128, 2048
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return PEAKS_FALLBACK, "fallback"
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,utilization.gpu")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) >= 10:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        busy = [r for r in rows if (num(r[9]) or 0) > 0] or rows
+        sm = [num(r[1]) for r in busy if num(r[1]) is not None]
+        reasons = set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in busy:
+            for name, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][2]),
+                "reasons": sorted(reasons), "samples": len(busy),
+                "power_w_max": max((num(r[3]) or 0) for r in busy)}
+
+
+# ------------------------------------------------------------ distributed --
+
+def dist_init(n_gpus: int):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus and world > 1:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    return rank, world, local
+
+
+def cpu_cores_used() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ oracle --
+
+def oracle_sample_inputs(rows: int, seed: int = 0):
+    """Host inputs for the CPU oracle: the layer's weights and `rows` sequences
+    with a (KV_LEN - 1)-token cache each."""
+    from invariant_numerics_b200 import synth
+    from oracle import reference as ref
+    p = host_layer_params(seed)
+    cache = ref.KVCache.empty(rows, HKV, KV_LEN, D)
+    for b in range(rows):
+        k = synth.kv_tensor(KV_LEN - 1, HKV, D, seed=seed + 100, stream=b)
+        v = synth.kv_tensor(KV_LEN - 1, HKV, D, seed=seed + 200, stream=b)
+        pos = np.arange(KV_LEN - 1)
+        cache.write("k", k, np.full(KV_LEN - 1, b), pos)
+        cache.write("v", v, np.full(KV_LEN - 1, b), pos)
+    x = synth.normal((rows, H), seed=seed + 300)
+    return p, cache, x
+
+
+_PARAMS = {}
+
+
+def host_layer_params(seed: int = 0):
+    if seed in _PARAMS:
+        return _PARAMS[seed]
+    from invariant_numerics_b200 import synth
+    from oracle import reference as ref
+    s = lambda i, shape: synth.normal(shape, seed=seed, stream=i, std=0.02)
+    p = ref.LayerParams(wq=s(1, (H, HQ * D)), wk=s(2, (H, HKV * D)), wv=s(3, (H, HKV * D)), wo=s(4, (HQ * D, H)),
+                        w_gate=s(5, (H, F)), w_up=s(6, (H, F)), w_down=s(7, (F, H)),
+                        g_attn=synth.uniform(H, seed=seed, stream=8, lo=0.5, hi=1.5),
+                        g_mlp=synth.uniform(H, seed=seed, stream=9, lo=0.5, hi=1.5),
+                        n_heads=HQ, n_kv_heads=HKV, head_dim=D)
+    _PARAMS[seed] = p
+    return p
+
+
+def time_oracle(rows: int, min_seconds: float, max_calls: int = 1000):
+    """Run the oracle decode layer on `rows` sequences until min_seconds pass."""
+    from oracle import reference as ref
+    p, cache, x = oracle_sample_inputs(rows)
+    slot = np.arange(rows)
+    pos = np.full(rows, KV_LEN - 1)
+    calls, t0 = 0, time.perf_counter()
+    while True:
+        ref.decode_layer(p, cache, x, slot, pos)
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or calls >= max_calls:
+            break
+    return rows * calls / el, el, calls
+
+
+# ------------------------------------------------------------------- ours --
+
+def build_gpu_layer(inv, torch, device):
+    p = host_layer_params(0)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    cfg = inv.LayerConfig(hidden=H, n_heads=HQ, n_kv_heads=HKV, ffn=F, max_pos=KV_LEN)
+    w = inv.LayerWeights(cfg, t(p.wq), t(p.wk), t(p.wv), t(p.wo), t(p.w_gate), t(p.w_up), t(p.w_down),
+                         t(p.g_attn), t(p.g_mlp))
+    return cfg, w
+
+
+def fill_cache(inv, torch, cache, n_tokens: int, seed: int):
+    """Synthetic K/V for positions 0..n_tokens-1 of every slot, quantised by
+    kv_quant_int16 (K/V ~ N(0,1) times a per-channel LogUniform(0.1, 10) factor)."""
+    from invariant_numerics_b200 import synth
+    dev = cache.k.device
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    scale = torch.from_numpy(synth.channel_scale(HKV, D, seed=seed)).to(dev)
+    chunk = 512
+    for s in range(cache.n_slots):
+        for p0 in range(0, n_tokens, chunk):
+            n = min(chunk, n_tokens - p0)
+            slot = torch.full((n,), s, dtype=torch.int32, device=dev)
+            pos = torch.arange(p0, p0 + n, dtype=torch.int32, device=dev)
+            for which in ("k", "v"):
+                x = torch.randn((n, HKV, D), generator=g, device=dev) * scale
+                inv.kv_quant_int16(x.contiguous(), slot, pos, cache, which)
+
+
+def layer_bytes(B, L):
+    """Algorithmic HBM bytes of one decode-layer step and of its kernels."""
+    Nqkv = (HQ + 2 * HKV) * D
+    gemm = {  # packed weights (4 B / weight) + A hi/lo (4 B / element) + y fp32 (+ residual fp32)
+        "gemm_qkv": 4 * H * Nqkv + 4 * B * H + 4 * B * Nqkv,
+        "gemm_o": 4 * HQ * D * H + 4 * B * HQ * D + 8 * B * H,
+        "gemm_gate_up": 4 * H * 2 * F + 4 * B * H + 4 * B * 2 * F,
+        "gemm_down": 4 * F * H + 4 * B * F + 8 * B * H,
+    }
+    S = (L + 255) // 256
+    attn_split = B * L * HKV * (2 * 2 * D + 2 * 4) + B * HQ * D * 4 + B * HQ * S * (D + 2) * 4
+    return gemm, attn_split
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    from invariant_numerics_b200 import build as _b
+    if rank == 0:
+        _b.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=device, timeout=__import__("datetime").timedelta(seconds=300))
+        dist.barrier()
+        _b.build()  # no-op once rank 0 has built
+    from invariant_numerics_b200 import invnum as inv
+    from invariant_numerics_b200 import synth
+
+    peaks, peak_kind = load_peaks()
+    cfg, w = build_gpu_layer(inv, torch, device)
+    cache = inv.KVCache(n_slots=BATCH, n_kv_heads=HKV, max_len=KV_LEN, device=device)
+    fill_cache(inv, torch, cache, KV_LEN - 1, seed=1 + rank)
+    x = torch.from_numpy(synth.normal((BATCH, H), seed=2 + rank)).to(device)
+    slot = torch.from_numpy(synth.permutation(BATCH, seed=3 + rank).astype(np.int32)).to(device)
+    pos = torch.full((BATCH,), KV_LEN - 1, dtype=torch.int32, device=device)
+    y = torch.empty_like(x)
+    call = inv.DecodeLayerCall(cfg, w, cache, x, slot, pos, y)
+    stream = torch.cuda.current_stream()
+    assert inv.inv_get_device_status() == inv.INV_OK
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+
+    # ----- device-resident timed region, kernels traced with CUDA events
+    K = args.steps
+    nk = inv.DECODE_LAYER_KERNELS
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for _ in range(K)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for k in range(K):  # create the events outside the timed region
+        for e in evs[k]:
+            e.record()
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    start.record(stream)
+    for k in range(K):
+        inv.inv_trace_events(evs[k])
+        call()
+    end.record(stream)
+    end.synchronize()
+    t_wall = time.perf_counter() - t_wall0
+    inv.inv_trace_events(None)
+    # a short timed region (small --steps) gives the 100 ms clock sampler too
+    # few points: keep running the same step, untimed, until 1.5 s have passed
+    while time.perf_counter() - t_wall0 < 1.5:
+        call()
+        torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = start.elapsed_time(end) / K
+    ms = max_over_ranks(ms)
+    st = inv.inv_get_device_status()
+    if st != inv.INV_OK:
+        raise RuntimeError(f"device status {inv.status_string(st)}")
+    kern_ms = {name: statistics.fmean(evs[k][2 * i].elapsed_time(evs[k][2 * i + 1]) for k in range(K))
+               for i, name in enumerate(inv.DECODE_LAYER_KERNEL_NAMES)}
+
+    # ----- end to end through the C ABI with host buffers
+    x_host = x.cpu().pin_memory()
+    slot_host = slot.cpu().pin_memory()
+    pos_host = pos.cpu().pin_memory()
+    y_host = torch.empty_like(x_host).pin_memory()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(K):
+        x.copy_(x_host, non_blocking=True)
+        slot.copy_(slot_host, non_blocking=True)
+        pos.copy_(pos_host, non_blocking=True)
+        call()
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    e1.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / K)
+    h2d = x_host.numel() * 4 + slot_host.numel() * 4 + pos_host.numel() * 4
+    d2h = y_host.numel() * 4
+
+    # ----- roofline of the dominant kernel (the attention split kernel)
+    gemm_b, attn_b = layer_bytes(BATCH, KV_LEN)
+    hbm = peaks["hbm_gbs"]
+    attn_gbs = attn_b / (kern_ms["attn_split"] * 1e-3) / 1e9
+    kernels = {}
+    for name, t in kern_ms.items():
+        ent = {"us": round(t * 1e3, 2)}
+        if name in gemm_b:
+            ent["gbs"] = round(gemm_b[name] / (t * 1e-3) / 1e9, 1)
+            ent["frac_hbm"] = round(ent["gbs"] / hbm, 3)
+        if name == "attn_split":
+            ent["gbs"] = round(attn_gbs, 1)
+            ent["frac_hbm"] = round(attn_gbs / hbm, 3)
+        kernels[name] = ent
+    step_bytes = sum(gemm_b.values()) + attn_b
+    result = {
+        "metric": "batch-invariant decode-layer tokens/s",
+        "value": round(BATCH * world / (ms * 1e-3), 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16 hi/lo products, f32 accumulate; int16 KV",
+        "data": "synthetic",
+        "config": {"workload": f"decode_layer H{H} Hq{HQ} Hkv{HKV} D{D} F{F} B{BATCH} kv{KV_LEN}",
+                   "global_batch": BATCH * world, "seq_len": KV_LEN, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (708.8 MB packed weights + 1.09 GB INT16 KV per step)"},
+        "roofline": {"kernel": "attn_split", "bound": "hbm", "achieved": round(attn_gbs, 1), "peak": hbm,
+                     "unit": "GB/s", "frac": round(attn_gbs / hbm, 4), "traffic": None,
+                     "peak_source": f"{peak_kind} hbm_gbs",
+                     "algorithmic_bytes_per_launch": attn_b},
+        "step_roofline": {"bytes": step_bytes, "hbm_bound_ms": round(step_bytes / (hbm * 1e9) * 1e3, 4),
+                          "frac": round(step_bytes / (hbm * 1e9) * 1e3 / ms, 4)},
+        "kernels": kernels,
+        "e2e": {"value": round(BATCH * world / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": K * (nk + 0),
+        "clocks": clocks,
+        "wall_s_timed": round(t_wall, 3),
+    }
+
+    if not args.no_components and rank == 0:
+        result["components"] = bench_components(inv, torch, device, peaks, peak_kind)
+    if not args.no_cpu_baseline and rank == 0 and world == 1:
+        v, el, calls = time_oracle(args.oracle_rows, args.oracle_seconds)
+        result["cpu_baseline"] = {"value": round(v, 4), "unit": "tokens/s", "cores": cpu_cores_used(),
+                                  "kind": "oracle",
+                                  "sample": f"{args.oracle_rows} sequences x {calls} oracle decode_layer calls "
+                                            f"(same layer shape, kv {KV_LEN}), {el:.1f} s"}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def bench_components(inv, torch, device, peaks, peak_kind):
+    """Compensated GEMM (K 4096, N 4096/11008, M 1..1024) and decode attention
+    (32/8 heads, ragged lengths U(128, 8192), B 64), each timed per launch with
+    CUDA events, L2 flushed between launches."""
+    from invariant_numerics_b200 import synth
+    out = {}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    tc_peak = peaks["bf16_tflops"]
+
+    def timed(fn, reps=5):
+        ts = []
+        for r in range(reps + 2):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            if r >= 2:
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    K = 4096
+    A = torch.from_numpy(synth.normal_with_outliers((1024, K), seed=10)).to(device)
+    hi, lo = inv.heal_split(A)
+    gem = {}
+    for N in (4096, 11008):
+        W = torch.from_numpy(synth.normal((K, N), seed=11, std=0.02)).to(device)
+        P, e = inv.heal_pack_weight(W)
+        del W
+        for M in (1, 3, 17, 64, 256, 1024):
+            a_hi, a_lo = hi[:M].contiguous(), lo[:M].contiguous()
+            y = torch.empty((M, N), dtype=torch.float32, device=device)
+            t = timed(lambda: inv.comp_gemm(a_hi, a_lo, P, e, out=y))
+            useful = 2.0 * M * N * K / (t * 1e-3) / 1e12
+            byts = 4 * N * K + 4 * M * K + 4 * M * N
+            gbs = byts / (t * 1e-3) / 1e9
+            gem[f"M{M}_N{N}"] = {"us": round(t * 1e3, 2), "useful_tflops": round(useful, 2),
+                                 "frac_of_peak_over_3": round(useful / (tc_peak / 3), 4),
+                                 "gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    out["comp_gemm"] = {"shapes": gem, "peak_tflops": tc_peak, "peak_source": f"{peak_kind} bf16_tflops (fp16 = bf16 rate)",
+                        "target": ">= 0.5 x peak / 3 useful at M 256, 1024"}
+
+    B = 64
+    lens = synth.ragged_lengths(B, seed=40)
+    cache = inv.KVCache(n_slots=B, n_kv_heads=HKV, max_len=8192, device=device)
+    g = torch.Generator(device=device)
+    g.manual_seed(41)
+    for b in range(B):
+        L = int(lens[b])
+        sl = torch.full((L,), b, dtype=torch.int32, device=device)
+        ps = torch.arange(L, dtype=torch.int32, device=device)
+        for which in ("k", "v"):
+            inv.kv_quant_int16(torch.randn((L, HKV, D), generator=g, device=device), sl, ps, cache, which)
+    q = torch.from_numpy(synth.normal((B, HQ, D), seed=42)).to(device)
+    slot = torch.arange(B, dtype=torch.int32, device=device)
+    lens_d = torch.from_numpy(lens).to(device)
+    o = torch.empty_like(q)
+    ws = torch.empty(inv.attn_decode_workspace_size(B, HQ, 8192), dtype=torch.uint8, device=device)
+    t = timed(lambda: inv.attn_decode_fixedsplit(q, cache, slot, lens_d, 0.08838834764831845, out=o, workspace=ws))
+    S = (lens.astype(np.int64) + 255) // 256
+    byts = int(lens.astype(np.int64).sum()) * HKV * 520 + B * HQ * D * 4 * 2 + int(S.sum()) * HQ * (D + 2) * 4 * 2
+    gbs = byts / (t * 1e-3) / 1e9
+    out["attention"] = {"B": B, "mean_len": float(lens.mean()), "us": round(t * 1e3, 2), "gbs": round(gbs, 1),
+                        "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "bytes": byts,
+                        "note": "split + combine kernels, L2 flushed between launches"}
+    assert inv.inv_get_device_status() == inv.INV_OK
+    return out
+
+
+# -------------------------------------------------------------- reference --
+
+def run_reference(args, rank, world):
+    """The CPU oracle as it stands, on a bounded sample of the same workload."""
+    if rank != 0:
+        return
+    rows = args.oracle_rows
+    times = []
+    from oracle import reference as ref
+    p, cache, x = oracle_sample_inputs(rows)
+    slot = np.arange(rows)
+    pos = np.full(rows, KV_LEN - 1)
+    for _ in range(args.warmup):
+        ref.decode_layer(p, cache, x, slot, pos)
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        ref.decode_layer(p, cache, x, slot, pos)
+        times.append(time.perf_counter() - t0)
+    ms = statistics.fmean(times) * 1e3
+    v = rows / (ms * 1e-3)
+    sample = f"{rows} sequences per step (kv {KV_LEN}), float64 oracle decode_layer"
+    print(json.dumps({
+        "impl": "reference", "metric": "batch-invariant decode-layer tokens/s", "value": round(v, 4),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"decode_layer H{H} Hq{HQ} Hkv{HKV} D{D} F{F} B{BATCH} kv{KV_LEN}",
+                   "global_batch": BATCH * world, "seq_len": KV_LEN, "parallelism": "cpu oracle, rank 0"},
+        "cpu_baseline": {"value": round(v, 4), "unit": "tokens/s", "cores": cpu_cores_used(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(v, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-components", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=BATCH, help="sequences per GPU (profiling of smaller cases)")
+    ap.add_argument("--kv", type=int, default=KV_LEN, help="KV length per sequence, multiple of 64")
+    ap.add_argument("--oracle-rows", type=int, default=2)
+    ap.add_argument("--oracle-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    global BATCH, KV_LEN
+    BATCH, KV_LEN = args.batch, args.kv
+    if KV_LEN % 64 != 0 or KV_LEN < 64:
+        raise SystemExit("--kv must be a positive multiple of 64")
+    rank, world, local = dist_init(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

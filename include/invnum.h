@@ -99,6 +99,18 @@ INV_API int inv_set_wait_limit_ns(long long ns);
  */
 INV_API int inv_selftest_wait_timeout(long long wait_ns, inv_stream stream);
 
+/*
+ * Kernel tracing for decode_layer (profiling aid; off by default).  With
+ * events != NULL and n_events >= 2 * INV_DECODE_LAYER_KERNELS, every later
+ * decode_layer call records events[2i] before and events[2i+1] after its i-th
+ * kernel launch, on the call's stream (i: 0 rmsnorm, 1 qkv GEMM, 2 rotary +
+ * quantise, 3 attention splits, 4 attention combine, 5 output GEMM, 6 rmsnorm,
+ * 7 gate/up GEMM, 8 SwiGLU, 9 down GEMM).  events are cudaEvent_t handles the
+ * caller created and keeps alive.  NULL / 0 switches tracing off.  Host-global.
+ */
+#define INV_DECODE_LAYER_KERNELS 10
+INV_API int inv_trace_events(void** events, int n_events);
+
 /* ------------------------------------------------------------------------
  * heal_split -- [HEAL] section 2: split fp32 activations into the binary16
  * (hi, lo) pair used by the compensated product:

@@ -400,7 +400,7 @@ size_t attn_workspace_bytes(int B, int Hq, int max_len_bound) {
 
 int launch_attention(const float* q, int B, int Hq, const inv_kv_cache& c, const int32_t* slot, const int32_t* len,
                      int max_len_bound, float sigma, float* out, uint16_t* out_hi, uint16_t* out_lo, void* ws,
-                     cudaStream_t s) {
+                     cudaStream_t s, int trace_base) {
   if (B == 0) return INV_OK;
   const int S_max = splits_for(max_len_bound);
   float* part_o = static_cast<float*>(ws);
@@ -421,15 +421,19 @@ int launch_attention(const float* q, int B, int Hq, const inv_kv_cache& c, const
     g_attn_attr[dev] = true;
   }
   dim3 grid(S_max, c.n_kv_heads, B);
+  trace_record(2 * trace_base, s);
   attn_split_kernel<<<grid, THREADS, kAttnSmem, s>>>(tk, tv, q, c.k_scale, c.v_scale, slot, len, Hq, c.n_kv_heads,
                                                      c.n_slots, c.max_len, max_len_bound, S_max, sigma, part_o, part_ml,
                                                      status_ptr(), wait_limit_ns());
   INV_CHECK_LAUNCH();
+  trace_record(2 * trace_base + 1, s);
   const int64_t warps = (int64_t)B * Hq;
+  trace_record(2 * trace_base + 2, s);
   attn_combine_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(
       part_o, part_ml, len, B, Hq, S_max, max_len_bound, out, reinterpret_cast<__half*>(out_hi),
       reinterpret_cast<__half*>(out_lo), status_ptr());
   INV_CHECK_LAUNCH();
+  trace_record(2 * trace_base + 3, s);
   return INV_OK;
 }
 
@@ -465,7 +469,7 @@ int attn_decode_fixedsplit(const float* q, int B, int n_heads, const inv_kv_cach
   const int mlb = max_len_bound > 0 ? (max_len_bound < cache->max_len ? max_len_bound : cache->max_len) : cache->max_len;
   if (ws_bytes < inv::attn_workspace_bytes(B, n_heads, mlb)) return INV_ERR_WORKSPACE;
   return inv::launch_attention(q, B, n_heads, *cache, slot, len, mlb, softmax_scale, out, out_hi, out_lo, workspace,
-                               static_cast<cudaStream_t>(stream));
+                               static_cast<cudaStream_t>(stream), -1);
 }
 
 }  // extern "C"

@@ -22,6 +22,9 @@ namespace inv {
 int* status_ptr();
 // Wait bound in ns for kernels launched now.
 long long wait_limit_ns();
+// decode_layer kernel tracing (see inv_trace_events).
+void set_trace(void** events, int n);
+void trace_record(int slot, cudaStream_t s);
 // Number of SMs of the current device (cached).
 int sm_count();
 // cuTensorMapEncodeTiled through the runtime's driver entry point.

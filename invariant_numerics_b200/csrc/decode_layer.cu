@@ -116,26 +116,35 @@ int decode_layer(const inv_layer_config* cfg, const inv_layer_weights* w, const 
   const int H = cfg->hidden, F = cfg->ffn, Hq = cfg->n_heads, Hkv = cfg->n_kv_heads;
   const int QD = Hq * 128, NQKV = (Hq + 2 * Hkv) * 128;
 
+  // Kernel i is bracketed by trace slots 2i and 2i+1 (inv_trace_events).
+#define INV_TRACED(i, expr)         \
+  do {                              \
+    inv::trace_record(2 * (i), s);  \
+    INV_TRY(expr);                  \
+    inv::trace_record(2 * (i) + 1, s); \
+  } while (0)
   // 1. h = rmsnorm(x) -> hi/lo
-  INV_TRY(inv::launch_rmsnorm(x_in, w->g_attn, B, H, cfg->eps, nullptr, ws.h_hi, ws.h_lo, s));
+  INV_TRACED(0, inv::launch_rmsnorm(x_in, w->g_attn, B, H, cfg->eps, nullptr, ws.h_hi, ws.h_lo, s));
   // 2. qkv = h W_qkv
-  INV_TRY(inv::launch_comp_gemm(ws.h_hi, ws.h_lo, B, H, H, w->w_qkv, w->e_qkv, NQKV, ws.qkv, NQKV, nullptr, 0, s));
+  INV_TRACED(1, inv::launch_comp_gemm(ws.h_hi, ws.h_lo, B, H, H, w->w_qkv, w->e_qkv, NQKV, ws.qkv, NQKV, nullptr, 0, s));
   // 3. rotary embedding of q and k; k, v -> INT16 cache; len = pos + 1
-  INV_TRY(inv::launch_rope_quant(ws.qkv, B, Hq, *cache, slot, pos, w->rope_cos, w->rope_sin, cfg->max_pos, ws.q_rot,
-                                 ws.lens, s));
-  // 4-5. fixed-split attention + ordered combine -> o hi/lo
+  INV_TRACED(2, inv::launch_rope_quant(ws.qkv, B, Hq, *cache, slot, pos, w->rope_cos, w->rope_sin, cfg->max_pos,
+                                       ws.q_rot, ws.lens, s));
+  // 4-5. fixed-split attention + ordered combine -> o hi/lo (kernels 3 and 4)
   INV_TRY(inv::launch_attention(ws.q_rot, B, Hq, *cache, slot, ws.lens, mlb, cfg->softmax_scale, ws.o, ws.o_hi,
-                                ws.o_lo, ws.attn, s));
+                                ws.o_lo, ws.attn, s, 3));
   // 6. x1 = x + o W_o
-  INV_TRY(inv::launch_comp_gemm(ws.o_hi, ws.o_lo, B, QD, QD, w->w_o, w->e_o, H, ws.x1, H, x_in, H, s));
+  INV_TRACED(5, inv::launch_comp_gemm(ws.o_hi, ws.o_lo, B, QD, QD, w->w_o, w->e_o, H, ws.x1, H, x_in, H, s));
   // 7. h2 = rmsnorm(x1) -> hi/lo
-  INV_TRY(inv::launch_rmsnorm(ws.x1, w->g_mlp, B, H, cfg->eps, nullptr, ws.h2_hi, ws.h2_lo, s));
+  INV_TRACED(6, inv::launch_rmsnorm(ws.x1, w->g_mlp, B, H, cfg->eps, nullptr, ws.h2_hi, ws.h2_lo, s));
   // 8. [gate | up] = h2 W_gu
-  INV_TRY(inv::launch_comp_gemm(ws.h2_hi, ws.h2_lo, B, H, H, w->w_gu, w->e_gu, 2 * F, ws.gu, 2 * F, nullptr, 0, s));
+  INV_TRACED(7, inv::launch_comp_gemm(ws.h2_hi, ws.h2_lo, B, H, H, w->w_gu, w->e_gu, 2 * F, ws.gu, 2 * F, nullptr, 0,
+                                      s));
   // 9. a = silu(gate) * up -> hi/lo
-  INV_TRY(inv::launch_swiglu_split(ws.gu, B, F, ws.a_hi, ws.a_lo, s));
+  INV_TRACED(8, inv::launch_swiglu_split(ws.gu, B, F, ws.a_hi, ws.a_lo, s));
   // 10. out = x1 + a W_down
-  INV_TRY(inv::launch_comp_gemm(ws.a_hi, ws.a_lo, B, F, F, w->w_down, w->e_down, H, x_out, H, ws.x1, H, s));
+  INV_TRACED(9, inv::launch_comp_gemm(ws.a_hi, ws.a_lo, B, F, F, w->w_down, w->e_down, H, x_out, H, ws.x1, H, s));
+#undef INV_TRACED
   return INV_OK;
 }
 

@@ -27,6 +27,6 @@ int launch_comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int 
 size_t attn_workspace_bytes(int B, int Hq, int max_len_bound);
 int launch_attention(const float* q, int B, int Hq, const inv_kv_cache& c, const int32_t* slot, const int32_t* len,
                      int max_len_bound, float sigma, float* out, uint16_t* out_hi, uint16_t* out_lo, void* ws,
-                     cudaStream_t s);
+                     cudaStream_t s, int trace_base);  // trace_base < 0: no tracing
 
 }  // namespace inv

@@ -44,6 +44,21 @@ int* status_ptr() {
 
 long long wait_limit_ns() { return g_wait_ns.load(); }
 
+namespace {
+void** g_trace = nullptr;
+int g_trace_n = 0;
+}  // namespace
+
+void set_trace(void** events, int n) {
+  g_trace = events;
+  g_trace_n = n;
+}
+
+void trace_record(int slot, cudaStream_t s) {
+  if (g_trace != nullptr && slot >= 0 && slot < g_trace_n && g_trace[slot] != nullptr)
+    cudaEventRecord(static_cast<cudaEvent_t>(g_trace[slot]), s);
+}
+
 int sm_count() {
   const int d = current_device();
   if (d < 0) return 148;
@@ -128,6 +143,16 @@ int inv_get_device_status(int* status_out, inv_stream stream) {
   const int zero = 0;
   if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return INV_ERR_CUDA;
   *status_out = v;
+  return INV_OK;
+}
+
+int inv_trace_events(void** events, int n_events) {
+  if (events == nullptr || n_events <= 0) {
+    inv::set_trace(nullptr, 0);
+    return INV_OK;
+  }
+  if (n_events < 2 * INV_DECODE_LAYER_KERNELS) return INV_ERR_INVALID_ARG;
+  inv::set_trace(events, n_events);
   return INV_OK;
 }
 

@@ -57,6 +57,7 @@ _SIGS = {
     "inv_get_device_status": (_i, [C.POINTER(_i), _p]),
     "inv_set_wait_limit_ns": (_i, [C.c_longlong]),
     "inv_selftest_wait_timeout": (_i, [C.c_longlong, _p]),
+    "inv_trace_events": (_i, [C.POINTER(C.c_void_p), _i]),
     "heal_split": (_i, [_p, _i64, _i64, _i64, _p, _p, _i64, _p]),
     "heal_packed_weight_bytes": (_sz, [_i, _i]),
     "heal_pack_weight": (_i, [_p, _i, _i, _p, _sz, _p, _p]),
@@ -123,6 +124,24 @@ def inv_set_wait_limit_ns(ns: int) -> None:
 
 def inv_selftest_wait_timeout(wait_ns: int, stream=None) -> None:
     _check("inv_selftest_wait_timeout", lib.inv_selftest_wait_timeout(int(wait_ns), _stream(stream)))
+
+
+DECODE_LAYER_KERNELS = 10
+DECODE_LAYER_KERNEL_NAMES = ("rmsnorm_attn", "gemm_qkv", "rope_quant", "attn_split", "attn_combine", "gemm_o",
+                             "rmsnorm_mlp", "gemm_gate_up", "swiglu_split", "gemm_down")
+
+
+def inv_trace_events(events) -> None:
+    """Trace decode_layer kernels into torch.cuda.Event objects (2 per kernel), or None to stop."""
+    if events is None:
+        _check("inv_trace_events", lib.inv_trace_events(None, 0))
+        return
+    for e in events:  # torch creates the CUDA event lazily, on first record
+        if e.cuda_event == 0:
+            e.record()
+    handles = (C.c_void_p * len(events))(*[C.c_void_p(e.cuda_event) for e in events])
+    inv_trace_events._keep = handles  # the library keeps the pointer
+    _check("inv_trace_events", lib.inv_trace_events(handles, len(events)))
 
 
 # ----------------------------------------------------------- operations ------
@@ -329,3 +348,23 @@ def decode_layer(cfg: LayerConfig, w: LayerWeights, cache: KVCache, x, slot, pos
     _check("decode_layer", lib.decode_layer(C.byref(cs), C.byref(ws_), C.byref(cc), _ptr(x), _ptr(slot), _ptr(pos), B,
                                             mlb, _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)))
     return out
+
+
+class DecodeLayerCall:
+    """decode_layer with every argument marshalled once: calling it issues one
+    C call with fixed device buffers (x, slot, pos, out, workspace)."""
+
+    def __init__(self, cfg: LayerConfig, w: LayerWeights, cache: KVCache, x, slot, pos, out, max_len_bound=None):
+        _need(x, torch.float32, "x"), _need(slot, torch.int32, "slot"), _need(pos, torch.int32, "pos")
+        _need(out, torch.float32, "out")
+        self.B = x.shape[0]
+        self.mlb = cache.max_len if max_len_bound is None else int(max_len_bound)
+        self._cs, self._ws, self._cc = cfg.struct(), w.struct(), cache.struct()
+        nbytes = lib.decode_layer_workspace_size(C.byref(self._cs), self.B, min(self.mlb, cache.max_len))
+        self.workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=x.device)
+        self._keep = (cfg, w, cache, x, slot, pos, out)
+        self._args = (C.byref(self._cs), C.byref(self._ws), C.byref(self._cc), _ptr(x), _ptr(slot), _ptr(pos), self.B,
+                      self.mlb, _ptr(out), _ptr(self.workspace), self.workspace.numel())
+
+    def __call__(self, stream=None):
+        _check("decode_layer", lib.decode_layer(*self._args, _stream(stream)))
