@@ -500,6 +500,7 @@ def run_reference(args, rank, world):
 
 
 def main():
+    global BATCH, KV_LEN
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3000)
@@ -514,7 +515,6 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    global BATCH, KV_LEN
     BATCH, KV_LEN = args.batch, args.kv
     if KV_LEN % 64 != 0 or KV_LEN < 64:
         raise SystemExit("--kv must be a positive multiple of 64")
