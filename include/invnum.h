@@ -222,6 +222,28 @@ INV_API int attn_decode_fixedsplit(const float* q, int B, int n_heads, const inv
                            float softmax_scale, float* out, uint16_t* out_hi, uint16_t* out_lo,
                            void* workspace, size_t ws_bytes, inv_stream stream);
 
+/*
+ * attn_decode_fixedsplit_noalloc -- the same attention, numerically identical,
+ * for callers that cannot allocate device memory or pass a workspace (an
+ * embedding application that owns the whole device-memory budget, a plug-in
+ * without an allocator, a latency-critical path where an allocation may
+ * synchronise the device).  No counterpart on the pages: it is an interface
+ * variant only.  The split partials live in a file-scope device array of
+ * INV_NOALLOC_SCRATCH_BYTES on every GPU that loads the library, held until
+ * exit.  Calls needing more than that (attn_decode_workspace_size(B, n_heads,
+ * max_len_bound) > INV_NOALLOC_SCRATCH_BYTES) return INV_ERR_WORKSPACE and
+ * launch nothing.  The first call on a device looks the array's address up
+ * (with that device current); make it before any stream capture.  All calls on
+ * a device share the array, so calls that overlap on the GPU race; calls
+ * ordered on one stream do not.  Allocates nothing; arguments and other errors
+ * as attn_decode_fixedsplit.
+ */
+#define INV_NOALLOC_SCRATCH_BYTES (34u << 20)
+INV_API int attn_decode_fixedsplit_noalloc(const float* q, int B, int n_heads, const inv_kv_cache* cache,
+                                           const int32_t* slot, const int32_t* len, int max_len_bound, int split,
+                                           float softmax_scale, float* out, uint16_t* out_hi, uint16_t* out_lo,
+                                           inv_stream stream);
+
 /* ------------------------------------------------------------------------
  * rmsnorm_bi -- [BI] table row "RMSNorm": always the data-parallel strategy,
  * one CTA per row and one fixed reduction order per row:

@@ -66,6 +66,8 @@ _SIGS = {
     "attn_decode_workspace_size": (_sz, [_i, _i, _i]),
     "attn_decode_fixedsplit": (_i, [_p, _i, _i, C.POINTER(KVCacheStruct), _p, _p, _i, _i, _f, _p, _p, _p, _p,
                                     _sz, _p]),
+    "attn_decode_fixedsplit_noalloc": (_i, [_p, _i, _i, C.POINTER(KVCacheStruct), _p, _p, _i, _i, _f, _p, _p,
+                                            _p, _p]),
     "rmsnorm_bi": (_i, [_p, _p, _i64, _i, _f, _p, _p, _p, _p]),
     "decode_layer_workspace_size": (_sz, [C.POINTER(LayerConfigStruct), _i, _i]),
     "decode_layer": (_i, [C.POINTER(LayerConfigStruct), C.POINTER(LayerWeightsStruct), C.POINTER(KVCacheStruct),
@@ -239,6 +241,29 @@ def attn_decode_fixedsplit(q, cache: KVCache, slot, lens, softmax_scale, max_len
            lib.attn_decode_fixedsplit(_ptr(q), B, Hq, C.byref(cs), _ptr(slot), _ptr(lens), mlb, KV_SPLIT,
                                       float(softmax_scale), _ptr(out), _ptr(hi), _ptr(lo), _ptr(workspace),
                                       workspace.numel(), _stream(stream)))
+    return (out, hi, lo) if want_split else out
+
+
+NOALLOC_SCRATCH_BYTES = 34 << 20
+
+
+def attn_decode_fixedsplit_noalloc(q, cache: KVCache, slot, lens, softmax_scale, max_len_bound=None, out=None,
+                                   want_split=False, stream=None):
+    """attn_decode_fixedsplit without a workspace argument, for callers that
+    cannot allocate device memory: the library's own fixed 34 MiB device
+    array holds the split partials (see include/invnum.h for the limits).
+    `out` (and the hi/lo buffers when want_split) must then be passed in by
+    such a caller; this wrapper only allocates them when they are omitted."""
+    _need(q, torch.float32, "q"), _need(slot, torch.int32, "slot"), _need(lens, torch.int32, "lens")
+    B, Hq, D = q.shape
+    mlb = cache.max_len if max_len_bound is None else int(max_len_bound)
+    out = torch.empty_like(q) if out is None else _need(out, torch.float32, "out")
+    hi = torch.empty(q.shape, dtype=torch.float16, device=q.device) if want_split else None
+    lo = torch.empty(q.shape, dtype=torch.float16, device=q.device) if want_split else None
+    cs = cache.struct()
+    _check("attn_decode_fixedsplit_noalloc",
+           lib.attn_decode_fixedsplit_noalloc(_ptr(q), B, Hq, C.byref(cs), _ptr(slot), _ptr(lens), mlb, KV_SPLIT,
+                                              float(softmax_scale), _ptr(out), _ptr(hi), _ptr(lo), _stream(stream)))
     return (out, hi, lo) if want_split else out
 
 
