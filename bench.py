@@ -13,7 +13,8 @@ hi/lo binary16 image; the KV cache holds 2047 synthetic tokens per sequence
 and every step decodes position 2047 (2048 keys).  The rows come in a seeded
 shuffled order of the cache slots.
 
-Reported: tokens/s of the whole job (value), the device-resident step time,
+Reported: tokens/s of the whole job (value: the step replayed as a CUDA graph
+of the decode_layer call, inputs resident), the device-resident step time,
 an end-to-end figure through the C ABI with host buffers (H2D of the step's
 inputs and D2H of its output inside the timed region), per-kernel times from
 CUDA events recorded around every kernel inside the timed region, the
@@ -228,7 +229,7 @@ def layer_bytes(B, L):
     gemm = {  # packed weights (4 B / weight) + A hi/lo (4 B / element) + y fp32 (+ residual fp32)
         "gemm_qkv": 4 * H * Nqkv + 4 * B * H + 4 * B * Nqkv,
         "gemm_o": 4 * HQ * D * H + 4 * B * HQ * D + 8 * B * H,
-        "gemm_gate_up": 4 * H * 2 * F + 4 * B * H + 4 * B * 2 * F,
+        "gemm_gate_up_swiglu": 4 * H * 2 * F + 4 * B * H + 4 * B * F,
         "gemm_down": 4 * F * H + 4 * B * F + 8 * B * H,
     }
     S = (L + 255) // 256
@@ -278,36 +279,60 @@ def run_ours(args, rank, world, local):
         call()
     torch.cuda.synchronize()
 
-    # ----- device-resident timed region, kernels traced with CUDA events
-    K = args.steps
-    nk = inv.DECODE_LAYER_KERNELS
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for _ in range(K)]
+    # ----- the step as a CUDA graph: one decode_layer call (9 kernels) captured
+    # once; every launch argument (buffers, tensor maps) is fixed for the run
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph):
+        call()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.perf_counter()
+    g0.record(stream)
+    for k in range(args.steps):
+        graph.replay()
+    g1.record(stream)
+    g1.synchronize()
+    t_wall = time.perf_counter() - t_wall0
+    # a short timed region (small --steps) gives the 100 ms clock sampler too
+    # few points: keep replaying the same step, untimed, until 1.5 s have passed
+    while time.perf_counter() - t_wall0 < 1.5:
+        graph.replay()
+        torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = max_over_ranks(g0.elapsed_time(g1) / args.steps)
+
+    # ----- the same call without the graph, every kernel traced with CUDA events
+    K = args.steps
+    nk = inv.DECODE_LAYER_KERNELS
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for k in range(K):  # create the events outside the timed region
         for e in evs[k]:
             e.record()
     barrier()
     torch.cuda.synchronize()
-    t_wall0 = time.perf_counter()
     start.record(stream)
     for k in range(K):
         inv.inv_trace_events(evs[k])
         call()
     end.record(stream)
     end.synchronize()
-    t_wall = time.perf_counter() - t_wall0
     inv.inv_trace_events(None)
-    # a short timed region (small --steps) gives the 100 ms clock sampler too
-    # few points: keep running the same step, untimed, until 1.5 s have passed
-    while time.perf_counter() - t_wall0 < 1.5:
-        call()
-        torch.cuda.synchronize()
-    clocks = sampler.stop()
-    ms = start.elapsed_time(end) / K
-    ms = max_over_ranks(ms)
+    ms_traced = max_over_ranks(start.elapsed_time(end) / K)
     st = inv.inv_get_device_status()
     if st != inv.INV_OK:
         raise RuntimeError(f"device status {inv.status_string(st)}")
@@ -327,7 +352,7 @@ def run_ours(args, rank, world, local):
         x.copy_(x_host, non_blocking=True)
         slot.copy_(slot_host, non_blocking=True)
         pos.copy_(pos_host, non_blocking=True)
-        call()
+        graph.replay()
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
     e1.synchronize()
@@ -373,9 +398,10 @@ def run_ours(args, rank, world, local):
         "step_roofline": {"bytes": step_bytes, "hbm_bound_ms": round(step_bytes / (hbm * 1e9) * 1e3, 4),
                           "frac": round(step_bytes / (hbm * 1e9) * 1e3 / ms, 4)},
         "kernels": kernels,
+        "ms_per_step_without_graph": round(ms_traced, 4),
         "e2e": {"value": round(BATCH * world / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": K * (nk + 0),
+        "gpu_launches": K * nk,
         "clocks": clocks,
         "wall_s_timed": round(t_wall, 3),
     }

@@ -105,10 +105,10 @@ INV_API int inv_selftest_wait_timeout(long long wait_ns, inv_stream stream);
  * decode_layer call records events[2i] before and events[2i+1] after its i-th
  * kernel launch, on the call's stream (i: 0 rmsnorm, 1 qkv GEMM, 2 rotary +
  * quantise, 3 attention splits, 4 attention combine, 5 output GEMM, 6 rmsnorm,
- * 7 gate/up GEMM, 8 SwiGLU, 9 down GEMM).  events are cudaEvent_t handles the
+ * 7 gate/up GEMM with fused SwiGLU, 8 down GEMM).  events are cudaEvent_t handles the
  * caller created and keeps alive.  NULL / 0 switches tracing off.  Host-global.
  */
-#define INV_DECODE_LAYER_KERNELS 10
+#define INV_DECODE_LAYER_KERNELS 9
 INV_API int inv_trace_events(void** events, int n_events);
 
 /* ------------------------------------------------------------------------
@@ -270,8 +270,8 @@ INV_API int rmsnorm_bi(const float* x, const float* gamma, int64_t rows, int hid
  *   o  = attn_decode_fixedsplit(q, len = pos + 1)    -> hi/lo
  *   x1 = x + comp_gemm(o, W_o)
  *   h2 = rmsnorm_bi(x1, g_mlp)                       -> hi/lo
- *   gu = comp_gemm(h2, W_gu)                          (N = 2 F: gate cols, then up cols)
- *   a  = silu(gate) * up                              -> hi/lo
+ *   a  = silu(gate) * up, gate/up = h2 W_gu: one comp_gemm over N = 2 F whose
+ *        epilogue applies silu(g) * u = g / (1 + exp(-g)) * u  -> hi/lo
  *   out = x1 + comp_gemm(a, W_down)
  * Rows of one sequence at consecutive positions (a prefill chunk) are legal:
  * every row's K/V is in the cache before any row attends.
@@ -295,7 +295,9 @@ typedef struct {
 typedef struct {
   const uint16_t* w_qkv;  const int8_t* e_qkv;   /* packed [H x (Hq+2Hkv)128] */
   const uint16_t* w_o;    const int8_t* e_o;     /* packed [Hq 128 x H] */
-  const uint16_t* w_gu;   const int8_t* e_gu;    /* packed [H x 2F] */
+  const uint16_t* w_gu;   const int8_t* e_gu;    /* packed [H x 2F], columns interleaved in
+                                                    groups of 16: for j < F/32, h in {0, 1}:
+                                                    gate 32j+16h .. +15, then up 32j+16h .. +15 */
   const uint16_t* w_down; const int8_t* e_down;  /* packed [F x H] */
   const float* g_attn;    /* [H] */
   const float* g_mlp;     /* [H] */

@@ -350,19 +350,35 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o, const floa
   if (L >= 1 && L <= len_limit) {
     const int S = (L + SPLIT - 1) / SPLIT;
     const float2* ml = part_ml + wid * S_max;
+    const float4* po = reinterpret_cast<const float4*>(part_o + wid * S_max * 128) + lane;
     float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, ml[s].x);
+    for (int s0 = 0; s0 < S; s0 += 8) {  // exact max: order does not matter
+      float2 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = s0 + j < S ? ml[s0 + j] : make_float2(-INFINITY, 0.0f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) M = fmaxf(M, v[j].x);
+    }
     float l = 0.0f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < S; ++s) {
-      const float2 v = ml[s];
-      const float f = expf(__fsub_rn(v.x, M));
-      l = __fadd_rn(l, __fmul_rn(v.y, f));
-      const float4 po = reinterpret_cast<const float4*>(part_o + (wid * S_max + s) * 128)[lane];
-      acc.x = __fadd_rn(acc.x, __fmul_rn(po.x, f));
-      acc.y = __fadd_rn(acc.y, __fmul_rn(po.y, f));
-      acc.z = __fadd_rn(acc.z, __fmul_rn(po.z, f));
-      acc.w = __fadd_rn(acc.w, __fmul_rn(po.w, f));
+    for (int s0 = 0; s0 < S; s0 += 8) {  // splits folded in ascending order, 8 loads in flight
+      float2 v[8];
+      float4 o[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        v[j] = s0 + j < S ? ml[s0 + j] : make_float2(-INFINITY, 0.0f);
+        o[j] = s0 + j < S ? po[(s0 + j) * 32] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (s0 + j >= S) break;
+        const float f = expf(__fsub_rn(v[j].x, M));
+        l = __fadd_rn(l, __fmul_rn(v[j].y, f));
+        acc.x = __fadd_rn(acc.x, __fmul_rn(o[j].x, f));
+        acc.y = __fadd_rn(acc.y, __fmul_rn(o[j].y, f));
+        acc.z = __fadd_rn(acc.z, __fmul_rn(o[j].z, f));
+        acc.w = __fadd_rn(acc.w, __fmul_rn(o[j].w, f));
+      }
     }
     res = make_float4(__fdiv_rn(acc.x, l), __fdiv_rn(acc.y, l), __fdiv_rn(acc.z, l), __fdiv_rn(acc.w, l));
   }

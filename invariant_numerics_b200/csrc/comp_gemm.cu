@@ -19,10 +19,12 @@
 // core's internal accumulation, whatever K is.  Two group buffers (2 x 128
 // TMEM columns) let the MMAs of group g+1 overlap the drain of group g.
 //
-// Warp roles (320 threads): warp 0 = TMA producer, warp 1 = TMEM allocator +
-// MMA issuer, warps 2..9 = epilogue (warp w reads TMEM lanes 32*(w%4).., the
-// column half (w-2)/4).  Persistent grid over tiles ordered N-panel-major so a
-// wave of CTAs shares weight panels and the A rows stay in L2.
+// Warp roles (320 threads): warp 0 = TMA producer (4 stages of A_hi, A_lo and
+// the weight panel), warp 1 = TMEM allocator + MMA issuer, warps 2..9 =
+// epilogue (warp w reads TMEM lanes 32*(w%4).., the column half (w-2)/4).
+// For M < 128 only round_up(M, 8) A rows are loaded (the MMA's other rows hold
+// stale data and produce output rows that are never stored).  Persistent grid over tiles ordered
+// N-panel-major so a wave of CTAs shares weight panels and A stays in L2.
 #include "common.cuh"
 #include "internal.h"
 
@@ -58,8 +60,8 @@ constexpr size_t kSmemBytes = sizeof(GemmSmem) + 1024;
 __global__ void __launch_bounds__(THREADS, 1)
     comp_gemm_kernel(const __grid_constant__ CUtensorMap tm_ahi, const __grid_constant__ CUtensorMap tm_alo,
                      const __grid_constant__ CUtensorMap tm_w, const int8_t* __restrict__ col_exp, float* y,
-                     int64_t ld_y, const float* residual, int64_t ld_r, int M, int N, int K, int* status,
-                     long long wait_ns) {
+                     int64_t ld_y, const float* residual, int64_t ld_r, __half* gate_hi, __half* gate_lo,
+                     int64_t ld_g, int M, int N, int K, int box_rows, int* status, long long wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -94,6 +96,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
+      const uint32_t a_bytes = (uint32_t)box_rows * (BK * 2);  // one of A_hi / A_lo
       uint32_t stage = 0, phase = 0;
       uint32_t issued_mask = 0, last_phase_mask = 0;
       for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
@@ -101,7 +104,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int kb = 0; kb < nkb; ++kb) {
           if (!inv::mbar_wait(&sm.empty[stage], phase ^ 1u, wait_ns, abort_flag, status)) goto producer_done;
           uint8_t* st = sm.stage[stage];
-          inv::mbar_arrive_expect_tx(&sm.full[stage], STAGE_BYTES);
+          inv::mbar_arrive_expect_tx(&sm.full[stage], 2 * a_bytes + W_BYTES);
           inv::tma_load_2d(st, &tm_ahi, &sm.full[stage], kb * BK, mt * BM);
           inv::tma_load_2d(st + A_BYTES, &tm_alo, &sm.full[stage], kb * BK, mt * BM);
           inv::tma_load_2d(st + 2 * A_BYTES, &tm_w, &sm.full[stage], kb * BK, nt * 2 * BN);
@@ -190,7 +193,43 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       {
         const int row = mt * BM + quarter * 32 + lane;
-        if (row < M) {
+        if (row < M && gate_hi != nullptr) {
+          // Fused SwiGLU: this thread's 32 packed columns are 16 gate columns
+          // then the 16 matching up columns of outputs f0 .. f0+15.
+          const int col0 = nt * BN + half * 32;
+          const int f0 = nt * (BN / 2) + half * 16;
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const char4 e4 = *reinterpret_cast<const char4*>(col_exp + col0 + i);
+            const int ev[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float t = __fadd_rn(acc_h[i + j], __fmul_rn(acc_x[i + j], 0x1p-11f));
+              v[i + j] = __fmul_rn(t, inv::pow2f(-ev[j]));
+            }
+          }
+          uint32_t hw[8], lw[8];
+          bool bad = false;
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) {
+            __half h0, l0, h1, l1;
+            const float a0 = __fmul_rn(__fdiv_rn(v[i], __fadd_rn(1.0f, expf(-v[i]))), v[16 + i]);
+            const float a1 = __fmul_rn(__fdiv_rn(v[i + 1], __fadd_rn(1.0f, expf(-v[i + 1]))), v[17 + i]);
+            bad |= inv::f16_overflow(a0) | inv::f16_overflow(a1);
+            inv::split_hi_lo(a0, h0, l0);
+            inv::split_hi_lo(a1, h1, l1);
+            hw[i / 2] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
+            lw[i / 2] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
+          }
+          if (bad) inv::record_status(status, INV_ERR_RANGE);
+          uint4* gh = reinterpret_cast<uint4*>(gate_hi + (int64_t)row * ld_g + f0);
+          uint4* gl = reinterpret_cast<uint4*>(gate_lo + (int64_t)row * ld_g + f0);
+          gh[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          gh[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+          gl[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          gl[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+        } else if (row < M) {
           const int col0 = nt * BN + half * 32;
           float* yr = y + (int64_t)row * ld_y + col0;
           const float* rr = residual ? residual + (int64_t)row * ld_r + col0 : nullptr;
@@ -236,13 +275,23 @@ namespace inv {
 int launch_comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
                      const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
                      const float* residual, int64_t ld_r, cudaStream_t s) {
+  return launch_comp_gemm_ex(a_hi, a_lo, M, K, ld_a, w_packed, col_exp, N, y, ld_y, residual, ld_r, nullptr, nullptr,
+                             0, s);
+}
+
+int launch_comp_gemm_ex(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
+                        const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
+                        const float* residual, int64_t ld_r, uint16_t* gate_hi, uint16_t* gate_lo, int64_t ld_g,
+                        cudaStream_t s) {
   if (M == 0) return INV_OK;
+  // A rows per load: the whole 128-row tile, or only round_up(M, 8) when M < 128
+  const int box_rows = M < BM ? (int)((M + 7) / 8 * 8) : BM;
   CUtensorMap ta, tl, tw;
   int rc = make_tensor_map_2d(&ta, a_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)M,
-                              (uint64_t)ld_a * 2, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+                              (uint64_t)ld_a * 2, BK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != INV_OK) return rc;
   rc = make_tensor_map_2d(&tl, a_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)M, (uint64_t)ld_a * 2,
-                          BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+                          BK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != INV_OK) return rc;
   rc = make_tensor_map_2d(&tw, w_packed, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)N * 2,
                           (uint64_t)K * 2, BK, 2 * BN, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -257,8 +306,10 @@ int launch_comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int 
   }
   const int64_t tiles = ((M + BM - 1) / BM) * (N / BN);
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-  comp_gemm_kernel<<<grid, THREADS, kSmemBytes, s>>>(ta, tl, tw, col_exp, y, ld_y, residual, ld_r, (int)M, N, K,
-                                                     status_ptr(), wait_limit_ns());
+  comp_gemm_kernel<<<grid, THREADS, kSmemBytes, s>>>(ta, tl, tw, col_exp, y, ld_y, residual, ld_r,
+                                                     reinterpret_cast<__half*>(gate_hi),
+                                                     reinterpret_cast<__half*>(gate_lo), ld_g, (int)M, N, K,
+                                                     box_rows, status_ptr(), wait_limit_ns());
   INV_CHECK_LAUNCH();
   return INV_OK;
 }

@@ -22,7 +22,6 @@ struct LayerWs {
   uint16_t *o_hi, *o_lo;
   float* x1;
   uint16_t *h2_hi, *h2_lo;
-  float* gu;
   uint16_t *a_hi, *a_lo;
   size_t bytes;
 };
@@ -49,7 +48,6 @@ LayerWs carve(const inv_layer_config& c, int B, int mlb, uint8_t* base) {
   w.x1 = reinterpret_cast<float*>(take(B * H * 4));
   w.h2_hi = reinterpret_cast<uint16_t*>(take(B * H * 2));
   w.h2_lo = reinterpret_cast<uint16_t*>(take(B * H * 2));
-  w.gu = reinterpret_cast<float*>(take(B * 2 * F * 4));
   w.a_hi = reinterpret_cast<uint16_t*>(take(B * F * 2));
   w.a_lo = reinterpret_cast<uint16_t*>(take(B * F * 2));
   w.bytes = off;
@@ -137,13 +135,11 @@ int decode_layer(const inv_layer_config* cfg, const inv_layer_weights* w, const 
   INV_TRACED(5, inv::launch_comp_gemm(ws.o_hi, ws.o_lo, B, QD, QD, w->w_o, w->e_o, H, ws.x1, H, x_in, H, s));
   // 7. h2 = rmsnorm(x1) -> hi/lo
   INV_TRACED(6, inv::launch_rmsnorm(ws.x1, w->g_mlp, B, H, cfg->eps, nullptr, ws.h2_hi, ws.h2_lo, s));
-  // 8. [gate | up] = h2 W_gu
-  INV_TRACED(7, inv::launch_comp_gemm(ws.h2_hi, ws.h2_lo, B, H, H, w->w_gu, w->e_gu, 2 * F, ws.gu, 2 * F, nullptr, 0,
-                                      s));
-  // 9. a = silu(gate) * up -> hi/lo
-  INV_TRACED(8, inv::launch_swiglu_split(ws.gu, B, F, ws.a_hi, ws.a_lo, s));
+  // 8-9. [gate | up] = h2 W_gu with the SwiGLU a = silu(gate) * up fused in the epilogue -> hi/lo
+  INV_TRACED(7, inv::launch_comp_gemm_ex(ws.h2_hi, ws.h2_lo, B, H, H, w->w_gu, w->e_gu, 2 * F, nullptr, 0, nullptr, 0,
+                                         ws.a_hi, ws.a_lo, F, s));
   // 10. out = x1 + a W_down
-  INV_TRACED(9, inv::launch_comp_gemm(ws.a_hi, ws.a_lo, B, F, F, w->w_down, w->e_down, H, x_out, H, ws.x1, H, s));
+  INV_TRACED(8, inv::launch_comp_gemm(ws.a_hi, ws.a_lo, B, F, F, w->w_down, w->e_down, H, x_out, H, ws.x1, H, s));
 #undef INV_TRACED
   return INV_OK;
 }

@@ -1,7 +1,7 @@
 // Bandwidth-bound kernels of the decode step: the binary16 hi/lo split, the
 // offline weight packing, batch-invariant RMSNorm, the INT16 KV quantiser, and
-// the per-row glue of the layer (rotary embedding + quantisation, SwiGLU,
-// embedding gather, greedy argmax).  All use 128-bit coalesced accesses where
+// the per-row glue of the layer (rotary embedding + quantisation, embedding
+// gather, greedy argmax).  All use 128-bit coalesced accesses where
 // the layout allows and fixed, shape-independent reduction orders.
 #include "common.cuh"
 #include "internal.h"
@@ -169,6 +169,81 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* __re
   if (bad) record_status(status, INV_ERR_RANGE);
 }
 
+// Single-pass form for hidden <= 256 * 4 * VPT: each thread keeps its VPT
+// float4 chunks (the same chunks t, t+256, ... in the same order as above) in
+// registers, so x is read once.  Same reduction order, same result bits.
+template <int VPT>
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_reg_kernel(const float* __restrict__ x,
+                                                                    const float* __restrict__ gamma, int hidden,
+                                                                    float eps, float* __restrict__ y,
+                                                                    __half* __restrict__ yh, __half* __restrict__ yl,
+                                                                    int* status) {
+  __shared__ float warp_sum[kNormThreads / 32];
+  __shared__ float r_sh;
+  const int64_t row = blockIdx.x;
+  const float4* xr = reinterpret_cast<const float4*>(x + row * hidden);
+  const int n4 = hidden / 4;
+  const float4* g4 = reinterpret_cast<const float4*>(gamma);
+  float4 v[VPT], gv[VPT];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int i = threadIdx.x + j * kNormThreads;
+    v[j] = i < n4 ? xr[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    gv[j] = i < n4 ? g4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  float s = 0.0f;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    if (threadIdx.x + j * kNormThreads < n4) {
+      s = __fmaf_rn(v[j].x, v[j].x, s);
+      s = __fmaf_rn(v[j].y, v[j].y, s);
+      s = __fmaf_rn(v[j].z, v[j].z, s);
+      s = __fmaf_rn(v[j].w, v[j].w, s);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
+  if ((threadIdx.x & 31) == 0) warp_sum[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = warp_sum[0];
+    for (int w = 1; w < kNormThreads / 32; ++w) t = __fadd_rn(t, warp_sum[w]);
+    const float mean = __fdiv_rn(t, (float)hidden);
+    r_sh = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean, eps)));
+  }
+  __syncthreads();
+  const float r = r_sh;
+  bool bad = false;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int i = threadIdx.x + j * kNormThreads;
+    if (i >= n4) continue;
+    const float4 g = gv[j];
+    float4 o;
+    o.x = __fmul_rn(__fmul_rn(v[j].x, r), g.x);
+    o.y = __fmul_rn(__fmul_rn(v[j].y, r), g.y);
+    o.z = __fmul_rn(__fmul_rn(v[j].z, r), g.z);
+    o.w = __fmul_rn(__fmul_rn(v[j].w, r), g.w);
+    if (y) reinterpret_cast<float4*>(y + row * hidden)[i] = o;
+    if (yh) {
+      __half h[4], l[4];
+      split_hi_lo(o.x, h[0], l[0]);
+      split_hi_lo(o.y, h[1], l[1]);
+      split_hi_lo(o.z, h[2], l[2]);
+      split_hi_lo(o.w, h[3], l[3]);
+      bad |= inv::f16_overflow(o.x) | inv::f16_overflow(o.y) | inv::f16_overflow(o.z) | inv::f16_overflow(o.w);
+      uint2 hv, lv;
+      hv.x = (uint32_t)__half_as_ushort(h[0]) | ((uint32_t)__half_as_ushort(h[1]) << 16);
+      hv.y = (uint32_t)__half_as_ushort(h[2]) | ((uint32_t)__half_as_ushort(h[3]) << 16);
+      lv.x = (uint32_t)__half_as_ushort(l[0]) | ((uint32_t)__half_as_ushort(l[1]) << 16);
+      lv.y = (uint32_t)__half_as_ushort(l[2]) | ((uint32_t)__half_as_ushort(l[3]) << 16);
+      reinterpret_cast<uint2*>(yh + row * hidden)[i] = hv;
+      reinterpret_cast<uint2*>(yl + row * hidden)[i] = lv;
+    }
+  }
+  if (bad) record_status(status, INV_ERR_RANGE);
+}
+
 // ------------------------------------------------------------- quantiser ----
 
 // Quantise one (token, kv head) row of 128 values held as one float4 per lane.
@@ -273,38 +348,6 @@ __global__ void rope_quant_kernel(const float* __restrict__ qkv, int T, int Hq, 
   quant_store_row(v, (is_k ? c.k : c.v) + rowi * 128, (is_k ? c.k_scale : c.v_scale) + rowi, lane);
 }
 
-// a = silu(gate) * up = gate / (1 + exp(-gate)) * up, then the hi/lo split.
-// gu: [T][2F] (gate columns 0..F-1, up columns F..2F-1).
-__global__ void swiglu_split_kernel(const float* __restrict__ gu, int64_t T, int F, __half* __restrict__ ah,
-                                    __half* __restrict__ al, int* status) {
-  const int64_t f4 = F / 4;
-  const int64_t total = T * f4;
-  bool bad = false;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t t = i / f4, c = i - t * f4;
-    const float4 g = reinterpret_cast<const float4*>(gu + t * 2 * F)[c];
-    const float4 u = reinterpret_cast<const float4*>(gu + t * 2 * F + F)[c];
-    const float gv[4] = {g.x, g.y, g.z, g.w};
-    const float uv[4] = {u.x, u.y, u.z, u.w};
-    __half h[4], l[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float sg = __fdiv_rn(gv[j], __fadd_rn(1.0f, expf(-gv[j])));
-      const float a = __fmul_rn(sg, uv[j]);
-      bad |= inv::f16_overflow(a);
-      split_hi_lo(a, h[j], l[j]);
-    }
-    uint2 hv, lv;
-    hv.x = (uint32_t)__half_as_ushort(h[0]) | ((uint32_t)__half_as_ushort(h[1]) << 16);
-    hv.y = (uint32_t)__half_as_ushort(h[2]) | ((uint32_t)__half_as_ushort(h[3]) << 16);
-    lv.x = (uint32_t)__half_as_ushort(l[0]) | ((uint32_t)__half_as_ushort(l[1]) << 16);
-    lv.y = (uint32_t)__half_as_ushort(l[2]) | ((uint32_t)__half_as_ushort(l[3]) << 16);
-    reinterpret_cast<uint2*>(ah + t * F)[c] = hv;
-    reinterpret_cast<uint2*>(al + t * F)[c] = lv;
-  }
-  if (bad) record_status(status, INV_ERR_RANGE);
-}
-
 __global__ void embed_kernel(const float* __restrict__ table, int vocab, int hidden, const int32_t* __restrict__ ids,
                              int B, float* __restrict__ x, int* status) {
   const int b = blockIdx.x;
@@ -368,8 +411,19 @@ namespace inv {
 int launch_rmsnorm(const float* x, const float* gamma, int64_t rows, int hidden, float eps, float* y,
                    uint16_t* yh, uint16_t* yl, cudaStream_t s) {
   if (rows == 0) return INV_OK;
-  rmsnorm_kernel<<<(unsigned)rows, kNormThreads, 0, s>>>(x, gamma, hidden, eps, y, reinterpret_cast<__half*>(yh),
-                                                        reinterpret_cast<__half*>(yl), status_ptr());
+  __half* h = reinterpret_cast<__half*>(yh);
+  __half* l = reinterpret_cast<__half*>(yl);
+  const int n4 = hidden / 4;
+  if (n4 <= kNormThreads)
+    rmsnorm_reg_kernel<1><<<(unsigned)rows, kNormThreads, 0, s>>>(x, gamma, hidden, eps, y, h, l, status_ptr());
+  else if (n4 <= 2 * kNormThreads)
+    rmsnorm_reg_kernel<2><<<(unsigned)rows, kNormThreads, 0, s>>>(x, gamma, hidden, eps, y, h, l, status_ptr());
+  else if (n4 <= 4 * kNormThreads)
+    rmsnorm_reg_kernel<4><<<(unsigned)rows, kNormThreads, 0, s>>>(x, gamma, hidden, eps, y, h, l, status_ptr());
+  else if (n4 <= 8 * kNormThreads)
+    rmsnorm_reg_kernel<8><<<(unsigned)rows, kNormThreads, 0, s>>>(x, gamma, hidden, eps, y, h, l, status_ptr());
+  else
+    rmsnorm_kernel<<<(unsigned)rows, kNormThreads, 0, s>>>(x, gamma, hidden, eps, y, h, l, status_ptr());
   INV_CHECK_LAUNCH();
   return INV_OK;
 }
@@ -383,15 +437,6 @@ int launch_rope_quant(const float* qkv, int T, int Hq, const inv_kv_cache& c, co
   const int64_t blocks = (warps * 32 + threads - 1) / threads;
   rope_quant_kernel<<<(unsigned)blocks, threads, 0, s>>>(qkv, T, Hq, c, slot, pos, rope_cos, rope_sin, max_pos, q_out,
                                                         len_out, status_ptr());
-  INV_CHECK_LAUNCH();
-  return INV_OK;
-}
-
-int launch_swiglu_split(const float* gu, int64_t T, int F, uint16_t* ah, uint16_t* al, cudaStream_t s) {
-  if (T == 0) return INV_OK;
-  const int threads = 256;
-  swiglu_split_kernel<<<grid_for(T * (F / 4), threads), threads, 0, s>>>(
-      gu, T, F, reinterpret_cast<__half*>(ah), reinterpret_cast<__half*>(al), status_ptr());
   INV_CHECK_LAUNCH();
   return INV_OK;
 }

@@ -16,11 +16,19 @@ int launch_rope_quant(const float* qkv, int T, int Hq, const inv_kv_cache& c, co
                       const int32_t* pos, const float* rope_cos, const float* rope_sin, int max_pos, float* q_out,
                       int32_t* len_out, cudaStream_t s);
 
-int launch_swiglu_split(const float* gu, int64_t T, int F, uint16_t* ah, uint16_t* al, cudaStream_t s);
 
 int launch_comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
                      const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
                      const float* residual, int64_t ld_r, cudaStream_t s);
+
+// comp_gemm with the fused SwiGLU epilogue: the packed weight holds gate/up
+// columns interleaved in groups of 16 ([gate 16 | up 16] per 32 columns);
+// writes the hi/lo split of silu(gate) * up to gate_hi/gate_lo [M][ld_g]
+// (N/2 outputs per row) instead of y.
+int launch_comp_gemm_ex(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
+                        const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
+                        const float* residual, int64_t ld_r, uint16_t* gate_hi, uint16_t* gate_lo, int64_t ld_g,
+                        cudaStream_t s);
 
 // Workspace layout of the attention: partial (m, l) and partial o per
 // (row, head, split).

@@ -128,9 +128,9 @@ def inv_selftest_wait_timeout(wait_ns: int, stream=None) -> None:
     _check("inv_selftest_wait_timeout", lib.inv_selftest_wait_timeout(int(wait_ns), _stream(stream)))
 
 
-DECODE_LAYER_KERNELS = 10
+DECODE_LAYER_KERNELS = 9
 DECODE_LAYER_KERNEL_NAMES = ("rmsnorm_attn", "gemm_qkv", "rope_quant", "attn_split", "attn_combine", "gemm_o",
-                             "rmsnorm_mlp", "gemm_gate_up", "swiglu_split", "gemm_down")
+                             "rmsnorm_mlp", "gemm_gate_up_swiglu", "gemm_down")
 
 
 def inv_trace_events(events) -> None:
@@ -327,20 +327,33 @@ class LayerConfig:
                                  self.eps, self.softmax_scale)
 
 
+def gate_up_order(F: int, device) -> torch.Tensor:
+    """Column order of [gate | up] (2F columns) for the fused SwiGLU epilogue:
+    per 32 outputs j and half h, 16 gate columns then the 16 matching up columns."""
+    j = torch.arange(F // 32, device=device).view(-1, 1, 1, 1)
+    h = torch.arange(2, device=device).view(1, -1, 1, 1)
+    part = torch.arange(2, device=device).view(1, 1, -1, 1)
+    i = torch.arange(16, device=device).view(1, 1, 1, -1)
+    return (part * F + 32 * j + 16 * h + i).reshape(-1)
+
+
 class LayerWeights:
     """Packed weights of one layer, built on the device by heal_pack_weight.
 
     Inputs are fp32 CUDA tensors in y = x W orientation: wq [H, Hq*128],
     wk/wv [H, Hkv*128], wo [Hq*128, H], w_gate/w_up [H, F], w_down [F, H],
-    g_attn/g_mlp [H].  The fused projections concatenate columns
-    (q | k | v and gate | up) before packing; packing is per column, so this
-    does not change any column's numbers.
+    g_attn/g_mlp [H].  The fused projections gather columns before packing:
+    q | k | v, and gate/up interleaved in groups of 16 (gate 32j+16h..+15,
+    then up 32j+16h..+15) as the fused SwiGLU epilogue expects.  Packing is
+    per column, so reordering columns does not change any column's numbers.
     """
 
     def __init__(self, cfg: LayerConfig, wq, wk, wv, wo, w_gate, w_up, w_down, g_attn, g_mlp, rope=None):
         self.w_qkv, self.e_qkv = heal_pack_weight(torch.cat([wq, wk, wv], dim=1).contiguous())
         self.w_o, self.e_o = heal_pack_weight(wo.contiguous())
-        self.w_gu, self.e_gu = heal_pack_weight(torch.cat([w_gate, w_up], dim=1).contiguous())
+        F = w_gate.shape[1]
+        self.w_gu, self.e_gu = heal_pack_weight(torch.cat([w_gate, w_up], dim=1)[:, gate_up_order(F, w_gate.device)]
+                                                .contiguous())
         self.w_down, self.e_down = heal_pack_weight(w_down.contiguous())
         self.g_attn = g_attn.contiguous()
         self.g_mlp = g_mlp.contiguous()

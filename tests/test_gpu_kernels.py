@@ -63,7 +63,7 @@ def test_pack_weight_bit_exact(inv):
 
 # ------------------------------------------------------------- rmsnorm -------
 
-@pytest.mark.parametrize("hidden", [512, 4096, 68])
+@pytest.mark.parametrize("hidden", [512, 4096, 68, 8196])
 def test_rmsnorm_parity(inv, hidden):
     x = synth.normal((9, hidden), seed=hidden)
     x[3] *= 1e-3
@@ -149,6 +149,26 @@ def test_comp_gemm_tiny_config(inv):
     assert status() == inv.INV_OK
 
 
+def test_comp_gemm_invariance_across_row_placement(inv):
+    """Rows land in different tiles and tensor-memory lanes (and, for M < 128,
+    in a trimmed A box) depending on M and offset: a row's bits must not
+    depend on where it lands."""
+    K, N = 1024, 384
+    A = synth.normal_with_outliers((600, K), seed=13)
+    W = synth.normal((K, N), seed=14, std=0.02)
+    P, e = inv.heal_pack_weight(dev(W))
+    hi, lo = inv.heal_split(dev(A))
+    full = inv.comp_gemm(hi, lo, P, e)
+    assert rowwise_err(host(full), ref.gemm(A, W)).max() <= TOL
+    for M in (1, 7, 8, 9, 63, 64, 65, 127, 128, 129, 255, 256, 257, 511, 513):
+        y = inv.comp_gemm(hi[:M].contiguous(), lo[:M].contiguous(), P, e)
+        assert torch.equal(y.view(torch.int32), full[:M].view(torch.int32)), M
+    for off in (1, 64, 100):  # the same rows at other positions
+        y = inv.comp_gemm(hi[off:off + 130].contiguous(), lo[off:off + 130].contiguous(), P, e)
+        assert torch.equal(y.view(torch.int32), full[off:off + 130].view(torch.int32)), off
+    assert status() == inv.INV_OK
+
+
 @pytest.mark.parametrize("N", [4096, 11008])
 def test_comp_gemm_sweep_parity_and_invariance(inv, N):
     K = 4096
@@ -173,7 +193,7 @@ def test_comp_gemm_sweep_parity_and_invariance(inv, N):
 
 
 def test_comp_gemm_ragged_and_residual(inv):
-    M, K, N = 133, 320, 192
+    M, K, N = 133, 320, 256
     A = synth.normal((M, K), seed=20)
     W = synth.normal((K, N), seed=21, std=0.5)
     R = synth.normal((M, N), seed=22)
@@ -193,7 +213,7 @@ def test_comp_gemm_rejects_bad_shapes(inv):
     P = torch.zeros((1, 2, 64, 100), dtype=torch.float16, device="cuda")
     e = torch.zeros((64,), dtype=torch.int8, device="cuda")
     with pytest.raises(inv.InvError) as ei:
-        inv.comp_gemm(hi, hi, P, e)
+        inv.comp_gemm(hi, hi, P, e)       # K % 64 != 0
     assert ei.value.code == inv.INV_ERR_UNSUPPORTED_SHAPE
 
 
