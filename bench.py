@@ -120,13 +120,7 @@ class ClockSampler:
 
 # ------------------------------------------------------------ distributed --
 
-def dist_init(n_gpus: int):
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != n_gpus and world > 1:
-        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
-    return rank, world, local
+from invariant_numerics_b200 import replicas  # noqa: E402
 
 
 def cpu_cores_used() -> int:
@@ -244,10 +238,8 @@ def run_ours(args, rank, world, local):
     from invariant_numerics_b200 import build as _b
     if rank == 0:
         _b.build()
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", device_id=device, timeout=__import__("datetime").timedelta(seconds=300))
-        dist.barrier()
+    if replicas.init("nccl", device=device):
+        replicas.barrier()
         _b.build()  # no-op once rank 0 has built
     from invariant_numerics_b200 import invnum as inv
     from invariant_numerics_b200 import synth
@@ -255,25 +247,19 @@ def run_ours(args, rank, world, local):
     peaks, peak_kind = load_peaks()
     cfg, w = build_gpu_layer(inv, torch, device)
     cache = inv.KVCache(n_slots=BATCH, n_kv_heads=HKV, max_len=KV_LEN, device=device)
-    fill_cache(inv, torch, cache, KV_LEN - 1, seed=1 + rank)
-    x = torch.from_numpy(synth.normal((BATCH, H), seed=2 + rank)).to(device)
-    slot = torch.from_numpy(synth.permutation(BATCH, seed=3 + rank).astype(np.int32)).to(device)
+    fill_cache(inv, torch, cache, KV_LEN - 1, seed=replicas.replica_seed(1, rank))
+    x = torch.from_numpy(synth.normal((BATCH, H), seed=replicas.replica_seed(2, rank))).to(device)
+    slot = torch.from_numpy(synth.permutation(BATCH, seed=replicas.replica_seed(3, rank)).astype(np.int32)).to(device)
     pos = torch.full((BATCH,), KV_LEN - 1, dtype=torch.int32, device=device)
     y = torch.empty_like(x)
     call = inv.DecodeLayerCall(cfg, w, cache, x, slot, pos, y)
     stream = torch.cuda.current_stream()
     assert inv.inv_get_device_status() == inv.INV_OK
 
-    def barrier():
-        if world > 1:
-            torch.distributed.barrier()
+    barrier = replicas.barrier
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(v, device=device)
 
     for _ in range(args.warmup):
         call()
@@ -377,7 +363,7 @@ def run_ours(args, rank, world, local):
     step_bytes = sum(gemm_b.values()) + attn_b
     result = {
         "metric": "batch-invariant decode-layer tokens/s",
-        "value": round(BATCH * world / (ms * 1e-3), 1),
+        "value": round(replicas.job_throughput(BATCH, world, ms), 1),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": K,
@@ -399,7 +385,7 @@ def run_ours(args, rank, world, local):
                           "frac": round(step_bytes / (hbm * 1e9) * 1e3 / ms, 4)},
         "kernels": kernels,
         "ms_per_step_without_graph": round(ms_traced, 4),
-        "e2e": {"value": round(BATCH * world / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(replicas.job_throughput(BATCH, world, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": K * nk,
         "clocks": clocks,
@@ -414,9 +400,9 @@ def run_ours(args, rank, world, local):
                                   "kind": "oracle",
                                   "sample": f"{args.oracle_rows} sequences x {calls} oracle decode_layer calls "
                                             f"(same layer shape, kv {KV_LEN}), {el:.1f} s"}
-    if world > 1:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
+    replicas.barrier()
+    del graph
+    replicas.finalize()
     if rank == 0:
         print(json.dumps(result), flush=True)
 
@@ -526,7 +512,7 @@ def run_reference(args, rank, world):
 
 
 def main():
-    global BATCH, KV_LEN
+    global BATCH, KV_LEN, H, HQ, HKV, F
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3000)
@@ -534,6 +520,10 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--hidden", type=int, default=H)
+    ap.add_argument("--heads", type=int, default=HQ)
+    ap.add_argument("--kv-heads", type=int, default=HKV)
+    ap.add_argument("--ffn", type=int, default=F)
     ap.add_argument("--batch", type=int, default=BATCH, help="sequences per GPU (profiling of smaller cases)")
     ap.add_argument("--kv", type=int, default=KV_LEN, help="KV length per sequence, multiple of 64")
     ap.add_argument("--oracle-rows", type=int, default=2)
@@ -542,9 +532,12 @@ def main():
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     BATCH, KV_LEN = args.batch, args.kv
+    H, HQ, HKV, F = args.hidden, args.heads, args.kv_heads, args.ffn
     if KV_LEN % 64 != 0 or KV_LEN < 64:
         raise SystemExit("--kv must be a positive multiple of 64")
-    rank, world, local = dist_init(args.gpus)
+    rank, world, local = replicas.env_ranks()
+    if world > 1 and world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     if args.impl == "reference":
         run_reference(args, rank, world)
     else:
