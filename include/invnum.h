@@ -311,6 +311,24 @@ INV_API int decode_layer(const inv_layer_config* cfg, const inv_layer_weights* w
                  float* x_out, void* workspace, size_t ws_bytes, inv_stream stream);
 
 /* ------------------------------------------------------------------------
+ * prefill_layer -- decode_layer for T rows that are consecutive positions
+ * pos0 .. pos0+T-1 of the one sequence in `slot` (a prefill chunk).  Same
+ * steps and same per-row arithmetic as decode_layer; the attention loads each
+ * 256-key split once for every row that reaches it and runs the decode
+ * kernel's per-row code on it, so every output row (and the cache) is
+ * bit-identical to decode_layer on the same rows ([BI] table row "Attention":
+ * chunked prefill and decode must not change a row's reduction).
+ *   x_in, x_out : fp32 [T][hidden].  0 <= slot < n_slots; 0 <= pos0;
+ *   pos0 + T <= min(max_len_bound (or cache->max_len), cfg->max_pos).
+ *   workspace : >= prefill_layer_workspace_size(cfg, T, max_len_bound) bytes.
+ * Errors: as decode_layer.
+ * ------------------------------------------------------------------------ */
+INV_API size_t prefill_layer_workspace_size(const inv_layer_config* cfg, int T, int max_len_bound);
+INV_API int prefill_layer(const inv_layer_config* cfg, const inv_layer_weights* w, const inv_kv_cache* cache,
+                          const float* x_in, int slot, int pos0, int T, int max_len_bound, float* x_out,
+                          void* workspace, size_t ws_bytes, inv_stream stream);
+
+/* ------------------------------------------------------------------------
  * rope_tables -- model constants for the rotary embedding of decode_layer:
  *   cos_out[p][i] = fl32(cos(p theta_i)), sin_out[p][i] = fl32(sin(p theta_i)),
  *   theta_i = base^(-2i/128), i < 64, 0 <= p < max_pos, evaluated in double

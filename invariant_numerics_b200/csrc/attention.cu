@@ -37,17 +37,34 @@ constexpr int THREADS = 128;                 // 4 warps x 64 keys
 constexpr int BOX_BYTES = 64 * 64 * 2;       // 64 keys x 64 d x int16
 constexpr int CODE_BYTES = 8 * BOX_BYTES;    // 256 keys x 128 d
 
-struct __align__(1024) AttnSmem {
-  uint8_t codes[CODE_BYTES];   // K codes, then V codes, then the warp exchange of O
-  float ks[SPLIT];
-  float vs[SPLIT];
+// Per-CTA scratch for the reductions of one row of one split.
+struct RowScratch {
   float red_m[4][4];
   float red_l[4][4];
   float red_w[4][4];
+};
+
+struct __align__(1024) DecodeSmem {
+  uint8_t codes[CODE_BYTES];   // K codes, then V codes, then the warp exchange of O
+  float ks[SPLIT];
+  float vs[SPLIT];
+  RowScratch rs;
   uint64_t bar_k, bar_v;
   int abort;
 };
-constexpr size_t kAttnSmem = sizeof(AttnSmem) + 1024;
+constexpr size_t kDecodeSmem = sizeof(DecodeSmem) + 1024;
+
+struct __align__(1024) PrefillSmem {
+  uint8_t kcodes[CODE_BYTES];  // K and V of one split stay resident for every row
+  uint8_t vcodes[CODE_BYTES];
+  float xo[4 * 4 * 128];       // warp exchange of O
+  float ks[SPLIT];
+  float vs[SPLIT];
+  RowScratch rs;
+  uint64_t bar_kv;
+  int abort;
+};
+constexpr size_t kPrefillSmem = sizeof(PrefillSmem) + 1024;
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -97,48 +114,25 @@ __device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
   return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
 }
 
-__global__ void __launch_bounds__(THREADS, 3)
-    attn_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                      const float* __restrict__ q, const float* __restrict__ kscale, const float* __restrict__ vscale,
-                      const int32_t* __restrict__ slot, const int32_t* __restrict__ len, int Hq, int Hkv,
-                      int n_slots, int max_len, int len_limit, int S_max, float sigma, float* __restrict__ part_o,
-                      float2* __restrict__ part_ml, int* status, long long wait_ns) {
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int G = Hq / Hkv;
-  const int L = len[b], sl = slot[b];
-  if (L < 1 || L > len_limit || sl < 0 || sl >= n_slots) {
-    if (s == 0 && h == 0 && threadIdx.x == 0) record_status(status, INV_ERR_INVALID_ARG);
-    return;
-  }
-  const int key0 = s * SPLIT;
-  if (key0 >= L) return;
-  const int n = min(SPLIT, L - key0);
-  const int nbox = (n + 63) >> 6;
-  const int row0 = (int)(((int64_t)sl * Hkv + h) * max_len + key0);
-
-  extern __shared__ uint8_t smem_raw[];
-  AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+// One query row of one split: the whole per-row computation shared by the
+// decode and prefill kernels, so a (row, split) gives the same bits in both.
+//   qrow : fp32 q of the row's G query heads of this kv head ([G][128]).
+//   n    : valid keys of this row in the split (1..256); keys >= n are masked.
+//   kbase/vbase : shared addresses of the split's K / V codes (swizzled layout).
+//   ks/vs : shared scales (zero beyond the keys that were loaded).
+//   xo   : shared [4 warps][4 heads][128] exchange buffer (may alias the codes
+//          in the decode kernel: it is written only after the last V read).
+//   issue_v / wait_v : hooks around the first V access (decode kernel: load V
+//          into the K buffer once every warp is done with K).
+//   out_o/out_ml : this row's partials for head 0 of the group, split s.
+template <bool kReuse, class IssueV, class WaitV>
+__device__ __forceinline__ void split_row(const float* __restrict__ qrow, int G, int n, uint32_t kbase,
+                                          uint32_t vbase, const float* ks, const float* vs, RowScratch& rs,
+                                          float* xo, float sigma, float* __restrict__ out_o,
+                                          float2* __restrict__ out_ml, int64_t head_stride_o,
+                                          int64_t head_stride_ml, bool ok, int* status, IssueV issue_v,
+                                          WaitV wait_v) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
-  const uint32_t cbase = inv::smem_u32(sm.codes);
-
-  if (tid == 0) {
-    inv::mbar_init(&sm.bar_k, 1);
-    inv::mbar_init(&sm.bar_v, 1);
-    sm.abort = 0;
-    inv::fence_mbar_init();
-  }
-  __syncthreads();
-  if (tid == 0) {
-    inv::mbar_arrive_expect_tx(&sm.bar_k, nbox * 2 * BOX_BYTES);
-    for (int bx = 0; bx < nbox; ++bx) {
-      inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES, &tm_k, &sm.bar_k, 0, row0 + 64 * bx);
-      inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES + BOX_BYTES, &tm_k, &sm.bar_k, 64, row0 + 64 * bx);
-    }
-  }
-  for (int j = tid; j < SPLIT; j += THREADS) {
-    sm.ks[j] = j < n ? kscale[(int64_t)row0 + j] : 0.0f;
-    sm.vs[j] = j < n ? vscale[(int64_t)row0 + j] : 0.0f;
-  }
 
   // B fragments of S^T = K Q^T: column g is query head g/2 of the group, its
   // hi part for even g and lo part for odd g; rows k = d.
@@ -147,28 +141,23 @@ __global__ void __launch_bounds__(THREADS, 3)
     const int head = g >> 1;
     const bool lo = (g & 1) != 0;
     const bool valid = head < G;
-    const float* qh = q + ((int64_t)b * Hq + (int64_t)h * G + head) * 128;
+    const float* qh = qrow + head * 128;
     bool bad = false;
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
+    for (int ks_ = 0; ks_ < 8; ++ks_) {
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
-        const int d = 16 * ks + 2 * c + 8 * r;
+        const int d = 16 * ks_ + 2 * c + 8 * r;
         const float x0 = valid ? qh[d] : 0.0f, x1 = valid ? qh[d + 1] : 0.0f;
         __half h0, l0, h1, l1;
         inv::split_hi_lo(x0, h0, l0);
         inv::split_hi_lo(x1, h1, l1);
         bad |= inv::f16_overflow(x0) | inv::f16_overflow(x1);
-        qf[ks][r] = lo ? pack_half2(l0, l1) : pack_half2(h0, h1);
+        qf[ks_][r] = lo ? pack_half2(l0, l1) : pack_half2(h0, h1);
       }
     }
     if (bad) record_status(status, INV_ERR_RANGE);
   }
-  __syncthreads();  // scales visible
-
-  bool ok = true;
-  if (lane == 0) ok = inv::mbar_wait(&sm.bar_k, 0, wait_ns, &sm.abort, status);
-  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 
   // ---------------------------------------------------------------- scores --
   float tsc[4][2];
@@ -181,20 +170,20 @@ __global__ void __launch_bounds__(THREADS, 3)
       float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       const int lkey = kb + ((lane >> 3) & 1) * 8 + (lane & 7);
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
+      for (int ks_ = 0; ks_ < 8; ++ks_) {
         uint32_t a[4], ah[4], al[4];
-        ldsm_x4(code_addr(cbase, lkey, 16 * ks + (lane >> 4) * 8), a);
+        ldsm_x4(code_addr(kbase, lkey, 16 * ks_ + (lane >> 4) * 8), a);
 #pragma unroll
         for (int i = 0; i < 4; ++i) unpack_dual(a[i], ah[i], al[i]);
-        mma16816(acc, ah, qf[ks][0], qf[ks][1]);
-        mma16816(acc, al, qf[ks][0], qf[ks][1]);
+        mma16816(acc, ah, qf[ks_][0], qf[ks_][1]);
+        mma16816(acc, al, qf[ks_][0], qf[ks_][1]);
       }
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const int key = kb + g + 8 * r;
         // acc[2r] = q_hi . code / 256, acc[2r+1] = q_lo . code / 256 (head c)
         const float dot = __fmul_rn(__fadd_rn(acc[2 * r], __fmul_rn(acc[2 * r + 1], 0x1p-11f)), 256.0f);
-        const float t = __fmul_rn(__fmul_rn(dot, sm.ks[key]), sigma);
+        const float t = __fmul_rn(__fmul_rn(dot, ks[key]), sigma);
         tsc[mt][r] = key < n ? t : -INFINITY;
         mx = fmaxf(mx, tsc[mt][r]);
       }
@@ -203,22 +192,13 @@ __global__ void __launch_bounds__(THREADS, 3)
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-  if (g == 0) sm.red_m[warp][c] = mx;
-  inv::fence_proxy_async_smem();  // K reads (generic proxy) before the TMA overwrite (async proxy)
+  if (g == 0) rs.red_m[warp][c] = mx;
+  inv::fence_proxy_async_smem();  // K reads (generic proxy) before any TMA overwrite (async proxy)
   __syncthreads();
-
-  bool v_issued = false;
-  if (tid == 0 && ok) {
-    v_issued = true;
-    inv::mbar_arrive_expect_tx(&sm.bar_v, nbox * 2 * BOX_BYTES);
-    for (int bx = 0; bx < nbox; ++bx) {
-      inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES, &tm_v, &sm.bar_v, 0, row0 + 64 * bx);
-      inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES + BOX_BYTES, &tm_v, &sm.bar_v, 64, row0 + 64 * bx);
-    }
-  }
+  issue_v();
 
   // ---------------------------------------------------------------- softmax --
-  const float M = fmaxf(fmaxf(sm.red_m[0][c], sm.red_m[1][c]), fmaxf(sm.red_m[2][c], sm.red_m[3][c]));
+  const float M = fmaxf(fmaxf(rs.red_m[0][c], rs.red_m[1][c]), fmaxf(rs.red_m[2][c], rs.red_m[3][c]));
   float w[4][2];
   float lsum = 0.0f, wmax = 0.0f;
 #pragma unroll
@@ -228,7 +208,7 @@ __global__ void __launch_bounds__(THREADS, 3)
       const int key = warp * 64 + mt * 16 + g + 8 * r;
       const float p = tsc[mt][r] == -INFINITY ? 0.0f : expf(__fsub_rn(tsc[mt][r], M));
       lsum = __fadd_rn(lsum, p);
-      w[mt][r] = (key < n && p != 0.0f) ? __fmul_rn(p, sm.vs[key]) : 0.0f;
+      w[mt][r] = (key < n && p != 0.0f) ? __fmul_rn(p, vs[key]) : 0.0f;
       wmax = fmaxf(wmax, w[mt][r]);
     }
   }
@@ -239,14 +219,14 @@ __global__ void __launch_bounds__(THREADS, 3)
   wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, 8));
   wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, 16));
   if (g == 0) {
-    sm.red_l[warp][c] = lsum;
-    sm.red_w[warp][c] = wmax;
+    rs.red_l[warp][c] = lsum;
+    rs.red_w[warp][c] = wmax;
   }
   __syncthreads();
   // per-(split, head) exponent E: max_j w_j 2^E in [2^14, 2^15)
   int E = 0;
   {
-    const float wm = fmaxf(fmaxf(sm.red_w[0][c], sm.red_w[1][c]), fmaxf(sm.red_w[2][c], sm.red_w[3][c]));
+    const float wm = fmaxf(fmaxf(rs.red_w[0][c], rs.red_w[1][c]), fmaxf(rs.red_w[2][c], rs.red_w[3][c]));
     if (wm > 0.0f) {
       int ex;
       frexpf(wm, &ex);
@@ -266,8 +246,7 @@ __global__ void __launch_bounds__(THREADS, 3)
     pw_lo[mt] = pack_half2(l0, l1);
   }
 
-  if (lane == 0 && ok) ok = inv::mbar_wait(&sm.bar_v, 0, wait_ns, &sm.abort, status);
-  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  ok = wait_v(ok);
 
   // --------------------------------------------------------------- values --
   float o[8][4];
@@ -291,7 +270,7 @@ __global__ void __launch_bounds__(THREADS, 3)
 #pragma unroll
       for (int dt = 0; dt < 8; ++dt) {
         uint32_t a[4], ah[4], al[4];
-        ldsm_x4_t(code_addr(cbase, lkey, 16 * dt + ((lane >> 3) & 1) * 8), a);
+        ldsm_x4_t(code_addr(vbase, lkey, 16 * dt + ((lane >> 3) & 1) * 8), a);
 #pragma unroll
         for (int i = 0; i < 4; ++i) unpack_dual(a[i], ah[i], al[i]);
         mma16816(o[dt], ah, b0, b1);
@@ -300,8 +279,7 @@ __global__ void __launch_bounds__(THREADS, 3)
     }
   }
   // o[dt]: (d = 16dt + g, col 2c = w_hi head c), (d, col 2c+1 = w_lo), (d+8, ...)
-  __syncthreads();  // every warp is done reading V codes: reuse the buffer
-  float* xo = reinterpret_cast<float*>(sm.codes);  // [warp][head][128]
+  __syncthreads();  // every warp is done reading V codes (xo may alias them)
   const float unscale = inv::pow2f(-E);
 #pragma unroll
   for (int dt = 0; dt < 8; ++dt) {
@@ -318,22 +296,156 @@ __global__ void __launch_bounds__(THREADS, 3)
     v = __fadd_rn(v, xo[(1 * 4 + head) * 128 + d]);
     v = __fadd_rn(v, xo[(2 * 4 + head) * 128 + d]);
     v = __fadd_rn(v, xo[(3 * 4 + head) * 128 + d]);
-    part_o[(((int64_t)b * Hq + (int64_t)h * G + head) * S_max + s) * 128 + d] = v;
+    out_o[head * head_stride_o + d] = v;
   }
   if (tid < G) {
-    const float Mh = fmaxf(fmaxf(sm.red_m[0][tid], sm.red_m[1][tid]), fmaxf(sm.red_m[2][tid], sm.red_m[3][tid]));
-    float l = sm.red_l[0][tid];
-    l = __fadd_rn(l, sm.red_l[1][tid]);
-    l = __fadd_rn(l, sm.red_l[2][tid]);
-    l = __fadd_rn(l, sm.red_l[3][tid]);
-    part_ml[((int64_t)b * Hq + (int64_t)h * G + tid) * S_max + s] = make_float2(Mh, l);
+    const float Mh = fmaxf(fmaxf(rs.red_m[0][tid], rs.red_m[1][tid]), fmaxf(rs.red_m[2][tid], rs.red_m[3][tid]));
+    float l = rs.red_l[0][tid];
+    l = __fadd_rn(l, rs.red_l[1][tid]);
+    l = __fadd_rn(l, rs.red_l[2][tid]);
+    l = __fadd_rn(l, rs.red_l[3][tid]);
+    out_ml[tid * head_stride_ml] = make_float2(Mh, l);
   }
+  if (kReuse) __syncthreads();  // the scratch and xo are reused by the next row
+}
+
+// Decode: one CTA per (row b, kv head h, split s).
+__global__ void __launch_bounds__(THREADS, 3)
+    attn_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                      const float* __restrict__ q, const float* __restrict__ kscale, const float* __restrict__ vscale,
+                      const int32_t* __restrict__ slot, const int32_t* __restrict__ len, int Hq, int Hkv,
+                      int n_slots, int max_len, int len_limit, int S_max, float sigma, float* __restrict__ part_o,
+                      float2* __restrict__ part_ml, int* status, long long wait_ns) {
+  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int G = Hq / Hkv;
+  const int L = len[b], sl = slot[b];
+  if (L < 1 || L > len_limit || sl < 0 || sl >= n_slots) {
+    if (s == 0 && h == 0 && threadIdx.x == 0) record_status(status, INV_ERR_INVALID_ARG);
+    return;
+  }
+  const int key0 = s * SPLIT;
+  if (key0 >= L) return;
+  const int n = min(SPLIT, L - key0);
+  const int nbox = (n + 63) >> 6;
+  const int row0 = (int)(((int64_t)sl * Hkv + h) * max_len + key0);
+
+  extern __shared__ uint8_t smem_raw[];
+  DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint32_t cbase = inv::smem_u32(sm.codes);
+
+  if (tid == 0) {
+    inv::mbar_init(&sm.bar_k, 1);
+    inv::mbar_init(&sm.bar_v, 1);
+    sm.abort = 0;
+    inv::fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    inv::mbar_arrive_expect_tx(&sm.bar_k, nbox * 2 * BOX_BYTES);
+    for (int bx = 0; bx < nbox; ++bx) {
+      inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES, &tm_k, &sm.bar_k, 0, row0 + 64 * bx);
+      inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES + BOX_BYTES, &tm_k, &sm.bar_k, 64, row0 + 64 * bx);
+    }
+  }
+  for (int j = tid; j < SPLIT; j += THREADS) {
+    sm.ks[j] = j < n ? kscale[(int64_t)row0 + j] : 0.0f;
+    sm.vs[j] = j < n ? vscale[(int64_t)row0 + j] : 0.0f;
+  }
+  __syncthreads();  // scales visible
+
+  bool ok = true;
+  if (lane == 0) ok = inv::mbar_wait(&sm.bar_k, 0, wait_ns, &sm.abort, status);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+
+  bool v_issued = false;
+  const int64_t obase = (int64_t)b * Hq + (int64_t)h * G;
+  split_row<false>(
+      q + obase * 128, G, n, cbase, cbase, sm.ks, sm.vs, sm.rs, reinterpret_cast<float*>(sm.codes), sigma,
+      part_o + (obase * S_max + s) * 128, part_ml + obase * S_max + s, (int64_t)S_max * 128, (int64_t)S_max, ok,
+      status,
+      [&]() {  // every warp is done with K: bring V into the same buffer
+        if (tid == 0 && ok) {
+          v_issued = true;
+          inv::mbar_arrive_expect_tx(&sm.bar_v, nbox * 2 * BOX_BYTES);
+          for (int bx = 0; bx < nbox; ++bx) {
+            inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES, &tm_v, &sm.bar_v, 0, row0 + 64 * bx);
+            inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES + BOX_BYTES, &tm_v, &sm.bar_v, 64, row0 + 64 * bx);
+          }
+        }
+      },
+      [&](bool okv) {
+        if (lane == 0 && okv) okv = inv::mbar_wait(&sm.bar_v, 0, wait_ns, &sm.abort, status);
+        return __shfl_sync(0xffffffffu, okv ? 1 : 0, 0) != 0;
+      });
   // No copy may still be landing in this CTA's shared memory when it exits
   // (only possible after a timed-out wait; immediate otherwise).
   if (tid == 0) {
     inv::mbar_wait(&sm.bar_k, 0, wait_ns, nullptr, status);
     if (v_issued) inv::mbar_wait(&sm.bar_v, 0, wait_ns, nullptr, status);
   }
+}
+
+// Prefill: rows r = 0..T-1 of one sequence (slot sl) at positions p0 + r.
+// One CTA per (kv head h, split s, block of ROWS_PER_CTA rows): the split's K
+// and V are loaded once and every row of the block that reaches split s runs
+// split_row -- the decode kernel's per-row code -- on them.
+constexpr int ROWS_PER_CTA = 64;
+
+__global__ void __launch_bounds__(THREADS, 1)
+    attn_prefill_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                              const float* __restrict__ q, const float* __restrict__ kscale,
+                              const float* __restrict__ vscale, int sl, int p0, int T, int Hq, int Hkv, int max_len,
+                              int S_max, float sigma, float* __restrict__ part_o, float2* __restrict__ part_ml,
+                              int* status, long long wait_ns) {
+  const int s = blockIdx.x, h = blockIdx.y, rb = blockIdx.z;
+  const int G = Hq / Hkv;
+  const int key0 = s * SPLIT;
+  // rows of this block that reach split s: p0 + r + 1 > key0
+  const int r_first = max(rb * ROWS_PER_CTA, key0 - p0);
+  const int r_last = min(T, (rb + 1) * ROWS_PER_CTA) - 1;
+  if (r_first > r_last) return;
+  const int n_max = min(SPLIT, p0 + r_last + 1 - key0);
+  const int nbox = (n_max + 63) >> 6;
+  const int row0 = (int)(((int64_t)sl * Hkv + h) * max_len + key0);
+
+  extern __shared__ uint8_t smem_raw[];
+  PrefillSmem& sm = *reinterpret_cast<PrefillSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, lane = tid & 31;
+
+  if (tid == 0) {
+    inv::mbar_init(&sm.bar_kv, 1);
+    sm.abort = 0;
+    inv::fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    inv::mbar_arrive_expect_tx(&sm.bar_kv, 2 * nbox * 2 * BOX_BYTES);
+    for (int bx = 0; bx < nbox; ++bx) {
+      inv::tma_load_2d(sm.kcodes + bx * 2 * BOX_BYTES, &tm_k, &sm.bar_kv, 0, row0 + 64 * bx);
+      inv::tma_load_2d(sm.kcodes + bx * 2 * BOX_BYTES + BOX_BYTES, &tm_k, &sm.bar_kv, 64, row0 + 64 * bx);
+      inv::tma_load_2d(sm.vcodes + bx * 2 * BOX_BYTES, &tm_v, &sm.bar_kv, 0, row0 + 64 * bx);
+      inv::tma_load_2d(sm.vcodes + bx * 2 * BOX_BYTES + BOX_BYTES, &tm_v, &sm.bar_kv, 64, row0 + 64 * bx);
+    }
+  }
+  for (int j = tid; j < SPLIT; j += THREADS) {
+    sm.ks[j] = j < n_max ? kscale[(int64_t)row0 + j] : 0.0f;
+    sm.vs[j] = j < n_max ? vscale[(int64_t)row0 + j] : 0.0f;
+  }
+  __syncthreads();
+  bool ok = true;
+  if (lane == 0) ok = inv::mbar_wait(&sm.bar_kv, 0, wait_ns, &sm.abort, status);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+
+  const uint32_t kbase = inv::smem_u32(sm.kcodes), vbase = inv::smem_u32(sm.vcodes);
+  for (int r = r_first; r <= r_last; ++r) {
+    const int n = min(SPLIT, p0 + r + 1 - key0);
+    const int64_t obase = (int64_t)r * Hq + (int64_t)h * G;
+    split_row<true>(q + obase * 128, G, n, kbase, vbase, sm.ks, sm.vs, sm.rs, sm.xo, sigma,
+              part_o + (obase * S_max + s) * 128, part_ml + obase * S_max + s, (int64_t)S_max * 128,
+              (int64_t)S_max, ok, status, []() {}, [](bool okv) { return okv; });
+  }
+  if (tid == 0) inv::mbar_wait(&sm.bar_kv, 0, wait_ns, nullptr, status);
 }
 
 // One warp per (row, head): fold splits s = 0, 1, ... in order.
@@ -402,6 +514,7 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o, const floa
 }
 
 bool g_attn_attr[64] = {};
+bool g_prefill_attr[64] = {};
 
 }  // namespace
 
@@ -431,14 +544,14 @@ int launch_attention(const float* q, int B, int Hq, const inv_kv_cache& c, const
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !g_attn_attr[dev]) {
-    if (cudaFuncSetAttribute(attn_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem) !=
+    if (cudaFuncSetAttribute(attn_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecodeSmem) !=
         cudaSuccess)
       return INV_ERR_CUDA;
     g_attn_attr[dev] = true;
   }
   dim3 grid(S_max, c.n_kv_heads, B);
   trace_record(2 * trace_base, s);
-  attn_split_kernel<<<grid, THREADS, kAttnSmem, s>>>(tk, tv, q, c.k_scale, c.v_scale, slot, len, Hq, c.n_kv_heads,
+  attn_split_kernel<<<grid, THREADS, kDecodeSmem, s>>>(tk, tv, q, c.k_scale, c.v_scale, slot, len, Hq, c.n_kv_heads,
                                                      c.n_slots, c.max_len, max_len_bound, S_max, sigma, part_o, part_ml,
                                                      status_ptr(), wait_limit_ns());
   INV_CHECK_LAUNCH();
@@ -447,6 +560,45 @@ int launch_attention(const float* q, int B, int Hq, const inv_kv_cache& c, const
   trace_record(2 * trace_base + 2, s);
   attn_combine_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(
       part_o, part_ml, len, B, Hq, S_max, max_len_bound, out, reinterpret_cast<__half*>(out_hi),
+      reinterpret_cast<__half*>(out_lo), status_ptr());
+  INV_CHECK_LAUNCH();
+  trace_record(2 * trace_base + 3, s);
+  return INV_OK;
+}
+
+int launch_attention_prefill(const float* q, int T, int Hq, const inv_kv_cache& c, int slot, int pos0,
+                             const int32_t* len, int max_len_bound, float sigma, float* out, uint16_t* out_hi,
+                             uint16_t* out_lo, void* ws, cudaStream_t s, int trace_base) {
+  if (T == 0) return INV_OK;
+  const int S_max = splits_for(max_len_bound);
+  float* part_o = static_cast<float*>(ws);
+  float2* part_ml = reinterpret_cast<float2*>(part_o + (size_t)T * Hq * S_max * 128);
+  const uint64_t rows = (uint64_t)c.n_slots * c.n_kv_heads * c.max_len;
+  CUtensorMap tk, tv;
+  int rc = make_tensor_map_2d(&tk, c.k, CU_TENSOR_MAP_DATA_TYPE_UINT16, 128, rows, 256, 64, 64,
+                              CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != INV_OK) return rc;
+  rc = make_tensor_map_2d(&tv, c.v, CU_TENSOR_MAP_DATA_TYPE_UINT16, 128, rows, 256, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != INV_OK) return rc;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !g_prefill_attr[dev]) {
+    if (cudaFuncSetAttribute(attn_prefill_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kPrefillSmem) != cudaSuccess)
+      return INV_ERR_CUDA;
+    g_prefill_attr[dev] = true;
+  }
+  dim3 grid(splits_for(pos0 + T), c.n_kv_heads, (T + ROWS_PER_CTA - 1) / ROWS_PER_CTA);
+  trace_record(2 * trace_base, s);
+  attn_prefill_split_kernel<<<grid, THREADS, kPrefillSmem, s>>>(tk, tv, q, c.k_scale, c.v_scale, slot, pos0, T, Hq,
+                                                                c.n_kv_heads, c.max_len, S_max, sigma, part_o,
+                                                                part_ml, status_ptr(), wait_limit_ns());
+  INV_CHECK_LAUNCH();
+  trace_record(2 * trace_base + 1, s);
+  const int64_t warps = (int64_t)T * Hq;
+  trace_record(2 * trace_base + 2, s);
+  attn_combine_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(
+      part_o, part_ml, len, T, Hq, S_max, max_len_bound, out, reinterpret_cast<__half*>(out_hi),
       reinterpret_cast<__half*>(out_lo), status_ptr());
   INV_CHECK_LAUNCH();
   trace_record(2 * trace_base + 3, s);

@@ -17,6 +17,8 @@ struct LayerWs {
   float* qkv;
   float* q_rot;
   int32_t* lens;
+  int32_t* rows_slot;  // prefill_layer: per-row slot / position arrays
+  int32_t* rows_pos;
   void* attn;
   float* o;
   uint16_t *o_hi, *o_lo;
@@ -41,6 +43,8 @@ LayerWs carve(const inv_layer_config& c, int B, int mlb, uint8_t* base) {
   w.qkv = reinterpret_cast<float*>(take(B * NQKV * 4));
   w.q_rot = reinterpret_cast<float*>(take(B * QD * 4));
   w.lens = reinterpret_cast<int32_t*>(take(B * 4));
+  w.rows_slot = reinterpret_cast<int32_t*>(take(B * 4));
+  w.rows_pos = reinterpret_cast<int32_t*>(take(B * 4));
   w.attn = take(inv::attn_workspace_bytes(B, c.n_heads, mlb));
   w.o = reinterpret_cast<float*>(take(B * QD * 4));
   w.o_hi = reinterpret_cast<uint16_t*>(take(B * QD * 2));
@@ -74,11 +78,63 @@ int bound_of(const inv_kv_cache* cache, int max_len_bound) {
   return max_len_bound > 0 ? (max_len_bound < cache->max_len ? max_len_bound : cache->max_len) : cache->max_len;
 }
 
+__global__ void fill_rows_kernel(int32_t* slot_out, int32_t* pos_out, int T, int slot, int pos0) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < T) {
+    slot_out[t] = slot;
+    pos_out[t] = pos0 + t;
+  }
+}
+
 #define INV_TRY(expr)          \
   do {                         \
     const int rc_ = (expr);    \
     if (rc_ != INV_OK) return rc_; \
   } while (0)
+
+// The layer's launches.  prefill_slot < 0: arbitrary rows (slot[b], pos[b]);
+// otherwise rows are positions prefill_pos0 + b of the sequence in
+// prefill_slot and the attention loads each split once for all of them.
+int run_layer(const inv_layer_config* cfg, const inv_layer_weights* w, const inv_kv_cache* cache, const float* x_in,
+              const int32_t* slot, const int32_t* pos, int B, int mlb, float* x_out, const LayerWs& ws,
+              cudaStream_t s, int prefill_slot, int prefill_pos0) {
+  const int H = cfg->hidden, F = cfg->ffn, Hq = cfg->n_heads, Hkv = cfg->n_kv_heads;
+  const int QD = Hq * 128, NQKV = (Hq + 2 * Hkv) * 128;
+
+  // Kernel i is bracketed by trace slots 2i and 2i+1 (inv_trace_events).
+#define INV_TRACED(i, expr)         \
+  do {                              \
+    inv::trace_record(2 * (i), s);  \
+    INV_TRY(expr);                  \
+    inv::trace_record(2 * (i) + 1, s); \
+  } while (0)
+  // 1. h = rmsnorm(x) -> hi/lo
+  INV_TRACED(0, inv::launch_rmsnorm(x_in, w->g_attn, B, H, cfg->eps, nullptr, ws.h_hi, ws.h_lo, s));
+  // 2. qkv = h W_qkv
+  INV_TRACED(1, inv::launch_comp_gemm(ws.h_hi, ws.h_lo, B, H, H, w->w_qkv, w->e_qkv, NQKV, ws.qkv, NQKV, nullptr, 0, s));
+  // 3. rotary embedding of q and k; k, v -> INT16 cache; len = pos + 1
+  INV_TRACED(2, inv::launch_rope_quant(ws.qkv, B, Hq, *cache, slot, pos, w->rope_cos, w->rope_sin, cfg->max_pos,
+                                       ws.q_rot, ws.lens, s));
+  // 4-5. fixed-split attention + ordered combine -> o hi/lo (kernels 3 and 4)
+  if (prefill_slot < 0) {
+    INV_TRY(inv::launch_attention(ws.q_rot, B, Hq, *cache, slot, ws.lens, mlb, cfg->softmax_scale, ws.o, ws.o_hi,
+                                  ws.o_lo, ws.attn, s, 3));
+  } else {
+    INV_TRY(inv::launch_attention_prefill(ws.q_rot, B, Hq, *cache, prefill_slot, prefill_pos0, ws.lens, mlb,
+                                          cfg->softmax_scale, ws.o, ws.o_hi, ws.o_lo, ws.attn, s, 3));
+  }
+  // 6. x1 = x + o W_o
+  INV_TRACED(5, inv::launch_comp_gemm(ws.o_hi, ws.o_lo, B, QD, QD, w->w_o, w->e_o, H, ws.x1, H, x_in, H, s));
+  // 7. h2 = rmsnorm(x1) -> hi/lo
+  INV_TRACED(6, inv::launch_rmsnorm(ws.x1, w->g_mlp, B, H, cfg->eps, nullptr, ws.h2_hi, ws.h2_lo, s));
+  // 8-9. [gate | up] = h2 W_gu with the SwiGLU a = silu(gate) * up fused in the epilogue -> hi/lo
+  INV_TRACED(7, inv::launch_comp_gemm_ex(ws.h2_hi, ws.h2_lo, B, H, H, w->w_gu, w->e_gu, 2 * F, nullptr, 0, nullptr, 0,
+                                         ws.a_hi, ws.a_lo, F, s));
+  // 10. out = x1 + a W_down
+  INV_TRACED(8, inv::launch_comp_gemm(ws.a_hi, ws.a_lo, B, F, F, w->w_down, w->e_down, H, x_out, H, ws.x1, H, s));
+#undef INV_TRACED
+  return INV_OK;
+}
 
 }  // namespace
 
@@ -110,38 +166,37 @@ int decode_layer(const inv_layer_config* cfg, const inv_layer_weights* w, const 
   const LayerWs ws = carve(*cfg, B, mlb, static_cast<uint8_t*>(workspace));
   if (ws_bytes < ws.bytes) return INV_ERR_WORKSPACE;
 
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int H = cfg->hidden, F = cfg->ffn, Hq = cfg->n_heads, Hkv = cfg->n_kv_heads;
-  const int QD = Hq * 128, NQKV = (Hq + 2 * Hkv) * 128;
+  return run_layer(cfg, w, cache, x_in, slot, pos, B, mlb, x_out, ws, static_cast<cudaStream_t>(stream), -1, 0);
+}
 
-  // Kernel i is bracketed by trace slots 2i and 2i+1 (inv_trace_events).
-#define INV_TRACED(i, expr)         \
-  do {                              \
-    inv::trace_record(2 * (i), s);  \
-    INV_TRY(expr);                  \
-    inv::trace_record(2 * (i) + 1, s); \
-  } while (0)
-  // 1. h = rmsnorm(x) -> hi/lo
-  INV_TRACED(0, inv::launch_rmsnorm(x_in, w->g_attn, B, H, cfg->eps, nullptr, ws.h_hi, ws.h_lo, s));
-  // 2. qkv = h W_qkv
-  INV_TRACED(1, inv::launch_comp_gemm(ws.h_hi, ws.h_lo, B, H, H, w->w_qkv, w->e_qkv, NQKV, ws.qkv, NQKV, nullptr, 0, s));
-  // 3. rotary embedding of q and k; k, v -> INT16 cache; len = pos + 1
-  INV_TRACED(2, inv::launch_rope_quant(ws.qkv, B, Hq, *cache, slot, pos, w->rope_cos, w->rope_sin, cfg->max_pos,
-                                       ws.q_rot, ws.lens, s));
-  // 4-5. fixed-split attention + ordered combine -> o hi/lo (kernels 3 and 4)
-  INV_TRY(inv::launch_attention(ws.q_rot, B, Hq, *cache, slot, ws.lens, mlb, cfg->softmax_scale, ws.o, ws.o_hi,
-                                ws.o_lo, ws.attn, s, 3));
-  // 6. x1 = x + o W_o
-  INV_TRACED(5, inv::launch_comp_gemm(ws.o_hi, ws.o_lo, B, QD, QD, w->w_o, w->e_o, H, ws.x1, H, x_in, H, s));
-  // 7. h2 = rmsnorm(x1) -> hi/lo
-  INV_TRACED(6, inv::launch_rmsnorm(ws.x1, w->g_mlp, B, H, cfg->eps, nullptr, ws.h2_hi, ws.h2_lo, s));
-  // 8-9. [gate | up] = h2 W_gu with the SwiGLU a = silu(gate) * up fused in the epilogue -> hi/lo
-  INV_TRACED(7, inv::launch_comp_gemm_ex(ws.h2_hi, ws.h2_lo, B, H, H, w->w_gu, w->e_gu, 2 * F, nullptr, 0, nullptr, 0,
-                                         ws.a_hi, ws.a_lo, F, s));
-  // 10. out = x1 + a W_down
-  INV_TRACED(8, inv::launch_comp_gemm(ws.a_hi, ws.a_lo, B, F, F, w->w_down, w->e_down, H, x_out, H, ws.x1, H, s));
-#undef INV_TRACED
-  return INV_OK;
+size_t prefill_layer_workspace_size(const inv_layer_config* cfg, int T, int max_len_bound) {
+  return decode_layer_workspace_size(cfg, T, max_len_bound);
+}
+
+int prefill_layer(const inv_layer_config* cfg, const inv_layer_weights* w, const inv_kv_cache* cache,
+                  const float* x_in, int slot, int pos0, int T, int max_len_bound, float* x_out, void* workspace,
+                  size_t ws_bytes, inv_stream stream) {
+  INV_TRY(validate(cfg, cache));
+  if (!w || T < 0 || slot < 0 || slot >= cache->n_slots || pos0 < 0) return INV_ERR_INVALID_ARG;
+  if (T == 0) return INV_OK;
+  if (T > 65535) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (!x_in || !x_out || !workspace || x_in == x_out) return INV_ERR_INVALID_ARG;
+  if (!w->w_qkv || !w->e_qkv || !w->w_o || !w->e_o || !w->w_gu || !w->e_gu || !w->w_down || !w->e_down ||
+      !w->g_attn || !w->g_mlp || !w->rope_cos || !w->rope_sin)
+    return INV_ERR_INVALID_ARG;
+  if (!cache->k || !cache->v || !cache->k_scale || !cache->v_scale) return INV_ERR_INVALID_ARG;
+  if (!inv::aligned16(x_in) || !inv::aligned16(x_out) || !inv::aligned16(workspace) || !inv::aligned16(w->rope_cos) ||
+      !inv::aligned16(w->rope_sin) || !inv::aligned16(w->g_attn) || !inv::aligned16(w->g_mlp) ||
+      !inv::aligned16(cache->k) || !inv::aligned16(cache->v))
+    return INV_ERR_INVALID_ARG;
+  const int mlb = bound_of(cache, max_len_bound);
+  if ((int64_t)pos0 + T > mlb || (int64_t)pos0 + T > cfg->max_pos) return INV_ERR_INVALID_ARG;
+  const LayerWs ws = carve(*cfg, T, mlb, static_cast<uint8_t*>(workspace));
+  if (ws_bytes < ws.bytes) return INV_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  fill_rows_kernel<<<(T + 255) / 256, 256, 0, s>>>(ws.rows_slot, ws.rows_pos, T, slot, pos0);
+  INV_CHECK_LAUNCH();
+  return run_layer(cfg, w, cache, x_in, ws.rows_slot, ws.rows_pos, T, mlb, x_out, ws, s, slot, pos0);
 }
 
 }  // extern "C"

@@ -37,4 +37,11 @@ int launch_attention(const float* q, int B, int Hq, const inv_kv_cache& c, const
                      int max_len_bound, float sigma, float* out, uint16_t* out_hi, uint16_t* out_lo, void* ws,
                      cudaStream_t s, int trace_base);  // trace_base < 0: no tracing
 
+// Prefill form: rows t = 0..T-1 are consecutive positions pos0 + t of the
+// sequence in `slot`; each split's K/V is loaded once for all rows that reach
+// it, and every (row, split) runs the decode kernel's per-row code.
+int launch_attention_prefill(const float* q, int T, int Hq, const inv_kv_cache& c, int slot, int pos0,
+                             const int32_t* len, int max_len_bound, float sigma, float* out, uint16_t* out_hi,
+                             uint16_t* out_lo, void* ws, cudaStream_t s, int trace_base);
+
 }  // namespace inv

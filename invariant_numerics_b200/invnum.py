@@ -72,6 +72,9 @@ _SIGS = {
     "decode_layer_workspace_size": (_sz, [C.POINTER(LayerConfigStruct), _i, _i]),
     "decode_layer": (_i, [C.POINTER(LayerConfigStruct), C.POINTER(LayerWeightsStruct), C.POINTER(KVCacheStruct),
                           _p, _p, _p, _i, _i, _p, _p, _sz, _p]),
+    "prefill_layer_workspace_size": (_sz, [C.POINTER(LayerConfigStruct), _i, _i]),
+    "prefill_layer": (_i, [C.POINTER(LayerConfigStruct), C.POINTER(LayerWeightsStruct), C.POINTER(KVCacheStruct),
+                           _p, _i, _i, _i, _i, _p, _p, _sz, _p]),
     "rope_tables": (_i, [_i, _d, _p, _p, _p]),
     "embed_gather": (_i, [_p, _i, _i, _p, _i, _p, _p]),
     "argmax_rows": (_i, [_p, _i, _i, _i64, _p, _p]),
@@ -385,6 +388,24 @@ def decode_layer(cfg: LayerConfig, w: LayerWeights, cache: KVCache, x, slot, pos
     out = torch.empty_like(x) if out is None else _need(out, torch.float32, "out")
     _check("decode_layer", lib.decode_layer(C.byref(cs), C.byref(ws_), C.byref(cc), _ptr(x), _ptr(slot), _ptr(pos), B,
                                             mlb, _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+def prefill_layer(cfg: LayerConfig, w: LayerWeights, cache: KVCache, x, slot: int, pos0: int, max_len_bound=None,
+                  out=None, workspace=None, stream=None):
+    """Rows x [T, H] at positions pos0 .. pos0+T-1 of the sequence in `slot`;
+    bit-identical per row to decode_layer, with each attention split loaded
+    once for the whole chunk."""
+    _need(x, torch.float32, "x")
+    T = x.shape[0]
+    mlb = cache.max_len if max_len_bound is None else int(max_len_bound)
+    cs, ws_, cc = cfg.struct(), w.struct(), cache.struct()
+    nbytes = lib.prefill_layer_workspace_size(C.byref(cs), T, min(mlb, cache.max_len))
+    if workspace is None:
+        workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=x.device)
+    out = torch.empty_like(x) if out is None else _need(out, torch.float32, "out")
+    _check("prefill_layer", lib.prefill_layer(C.byref(cs), C.byref(ws_), C.byref(cc), _ptr(x), int(slot), int(pos0),
+                                              T, mlb, _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)))
     return out
 
 

@@ -245,3 +245,61 @@ def test_embed_and_argmax(inv):
     bad = inv.embed_gather(dev(table), dev(np.array([0, V], np.int32)))
     assert status() == inv.INV_ERR_INVALID_ARG
     assert np.array_equal(host(bad)[1], np.zeros(Hs, np.float32))
+
+
+def test_stack_32_layers_8192_prompt_chunked_prefill_and_128_decode_steps(inv):
+    """The chunked-prefill configuration at full size: 32 layers of the 7B-like
+    layer, vocab 32000, a random 8192-token prompt.  One-shot prefill versus
+    512-token chunked prefill (prefill_layer), then 128 greedy decode steps
+    (decode_layer): every layer's hidden states and every token id must be
+    bit-identical.  Weights are drawn on the device (this checks the GPU path
+    against itself; the oracle comparison is the 4-layer test above)."""
+    n_layers, V, T, chunk, n_dec, max_len = 32, 32000, 8192, 512, 128, 8384
+    g = torch.Generator(device="cuda")
+    g.manual_seed(2024)
+    cfg = inv.LayerConfig(hidden=H, n_heads=HQ, n_kv_heads=HKV, ffn=F, max_pos=max_len)
+    rope = inv.rope_tables(max_len)
+    layers = []
+    for _ in range(n_layers):
+        r = lambda *s: torch.randn(s, generator=g, device="cuda") * 0.02
+        layers.append(inv.LayerWeights(cfg, r(H, HQ * D), r(H, HKV * D), r(H, HKV * D), r(HQ * D, H), r(H, F),
+                                       r(H, F), r(F, H), torch.rand(H, generator=g, device="cuda") + 0.5,
+                                       torch.rand(H, generator=g, device="cuda") + 0.5, rope=rope))
+    embed = torch.randn((V, H), generator=g, device="cuda") * 0.02
+    g_final = torch.rand(H, generator=g, device="cuda") + 0.5
+    lm_P, lm_e = inv.heal_pack_weight((torch.randn((H, V), generator=g, device="cuda") * 0.02).contiguous())
+    prompt = torch.from_numpy(synth.token_ids(T, V, seed=600)).cuda()
+
+    def head(x):
+        hi, lo = inv.rmsnorm_bi(x, g_final, 1e-6, want_y=False, want_split=True)
+        return inv.argmax_rows(inv.comp_gemm(hi, lo, lm_P, lm_e))
+
+    def run(chunked):
+        caches = [inv.KVCache(n_slots=1, n_kv_heads=HKV, max_len=max_len) for _ in range(n_layers)]
+        spans = [(a, min(T, a + chunk)) for a in range(0, T, chunk)] if chunked else [(0, T)]
+        last = None
+        for a, b in spans:
+            x = inv.embed_gather(embed, prompt[a:b].contiguous())
+            for l in range(n_layers):
+                x = inv.prefill_layer(cfg, layers[l], caches[l], x, 0, a)
+            last = x
+        ids = [int(head(last[-1:].contiguous())[0])]
+        dec_states = []
+        for t in range(n_dec):
+            x = inv.embed_gather(embed, torch.tensor([ids[-1]], dtype=torch.int32, device="cuda"))
+            for l in range(n_layers):
+                x = inv.decode_layer(cfg, layers[l], caches[l], x, torch.zeros(1, dtype=torch.int32, device="cuda"),
+                                     torch.tensor([T + t], dtype=torch.int32, device="cuda"))
+            dec_states.append(x[0].clone())
+            ids.append(int(head(x)[0]))
+        return caches, last, ids, torch.stack(dec_states)
+
+    c1, last1, ids1, dec1 = run(chunked=False)
+    c2, last2, ids2, dec2 = run(chunked=True)
+    assert status() == inv.INV_OK
+    assert torch.equal(last1.view(torch.int32)[-chunk:], last2.view(torch.int32))  # final layer, last chunk
+    for l in range(n_layers):                                                     # every layer's cache
+        assert torch.equal(c1[l].k, c2[l].k) and torch.equal(c1[l].v, c2[l].v), l
+        assert torch.equal(c1[l].k_scale, c2[l].k_scale) and torch.equal(c1[l].v_scale, c2[l].v_scale), l
+    assert ids1 == ids2
+    assert torch.equal(dec1.view(torch.int32), dec2.view(torch.int32))

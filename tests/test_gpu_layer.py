@@ -101,3 +101,25 @@ def test_chunked_prefill_matches_one_shot(inv):
     assert torch.equal(one.view(torch.int32), chunked.view(torch.int32))
     assert torch.equal(a.k, b.k) and torch.equal(a.v, b.v)
     assert torch.equal(a.k_scale, b.k_scale) and torch.equal(a.v_scale, b.v_scale)
+
+
+def test_prefill_layer_bit_identical_to_decode_layer(inv):
+    """The prefill form (splits loaded once per chunk) gives the decode form's
+    bits for every row and writes the same cache, for chunks that start and
+    end inside splits and row blocks."""
+    p, cfg, w = make_layer(inv, **SMALL, seed=3)
+    T0, T1, T2 = 300, 77, 430    # chunk boundaries off the 256-key and 64-row grids
+    xs = synth.normal((T0 + T1 + T2, SMALL["H"]), seed=11)
+    a = inv.KVCache(n_slots=2, n_kv_heads=2, max_len=1024)
+    b = inv.KVCache(n_slots=2, n_kv_heads=2, max_len=1024)
+    start = 0
+    for T in (T0, T1, T2):
+        x = dev(xs[start:start + T].copy())
+        pos = np.arange(start, start + T, dtype=np.int32)
+        y_dec = inv.decode_layer(cfg, w, a, x, dev(np.ones(T, np.int32)), dev(pos))
+        y_pre = inv.prefill_layer(cfg, w, b, x, 1, start)
+        assert torch.equal(y_dec.view(torch.int32), y_pre.view(torch.int32)), start
+        start += T
+    assert torch.equal(a.k, b.k) and torch.equal(a.v, b.v)
+    assert torch.equal(a.k_scale, b.k_scale) and torch.equal(a.v_scale, b.v_scale)
+    assert status() == inv.INV_OK
