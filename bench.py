@@ -46,6 +46,11 @@ sys.path.insert(0, ROOT)
 H, HQ, HKV, D, F = 4096, 32, 8, 128, 11008
 BATCH, KV_LEN = 128, 2048
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) of one attn_split launch per decoded row at KV length
+# 2048, from the ncu capture in profiles/attn_split_B32_kv2048.md (B = 32:
+# 273.22 MB read + 6.52 MB written), scaled by rows.  Set to None whenever the
+# kernel changes until it is captured again.
+ATTN_SPLIT_DRAM_BYTES_PER_ROW_KV2048 = (273.219840e6 + 6.519296e6) / 32
 
 
 def load_peaks():
@@ -192,7 +197,7 @@ def time_oracle(rows: int, min_seconds: float, max_calls: int = 1000):
 def build_gpu_layer(inv, torch, device):
     p = host_layer_params(0)
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
-    cfg = inv.LayerConfig(hidden=H, n_heads=HQ, n_kv_heads=HKV, ffn=F, max_pos=KV_LEN)
+    cfg = inv.LayerConfig(hidden=H, n_heads=HQ, n_kv_heads=HKV, ffn=F, max_pos=max(KV_LEN, 8192))
     w = inv.LayerWeights(cfg, t(p.wq), t(p.wk), t(p.wv), t(p.wo), t(p.w_gate), t(p.w_up), t(p.w_down),
                          t(p.g_attn), t(p.g_mlp))
     return cfg, w
@@ -378,7 +383,10 @@ def run_ours(args, rank, world, local):
                    "global_batch": BATCH * world, "seq_len": KV_LEN, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (708.8 MB packed weights + 1.09 GB INT16 KV per step)"},
         "roofline": {"kernel": "attn_split", "bound": "hbm", "achieved": round(attn_gbs, 1), "peak": hbm,
-                     "unit": "GB/s", "frac": round(attn_gbs / hbm, 4), "traffic": None,
+                     "unit": "GB/s", "frac": round(attn_gbs / hbm, 4),
+                     "traffic": (round(ATTN_SPLIT_DRAM_BYTES_PER_ROW_KV2048 * BATCH)
+                                 if (KV_LEN == 2048 and ATTN_SPLIT_DRAM_BYTES_PER_ROW_KV2048) else None),
+                     "traffic_source": "ncu dram__bytes_read+write of a B=32 capture, scaled by rows",
                      "peak_source": f"{peak_kind} hbm_gbs",
                      "algorithmic_bytes_per_launch": attn_b},
         "step_roofline": {"bytes": step_bytes, "hbm_bound_ms": round(step_bytes / (hbm * 1e9) * 1e3, 4),
@@ -394,6 +402,7 @@ def run_ours(args, rank, world, local):
 
     if not args.no_components and rank == 0:
         result["components"] = bench_components(inv, torch, device, peaks, peak_kind)
+        result["components"]["prefill"] = bench_prefill(inv, torch, device, cfg, w)
     if not args.no_cpu_baseline and rank == 0 and world == 1:
         v, el, calls = time_oracle(args.oracle_rows, args.oracle_seconds)
         result["cpu_baseline"] = {"value": round(v, 4), "unit": "tokens/s", "cores": cpu_cores_used(),
@@ -474,6 +483,38 @@ def bench_components(inv, torch, device, peaks, peak_kind):
                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "bytes": byts,
                         "note": "split + combine kernels, L2 flushed between launches"}
     assert inv.inv_get_device_status() == inv.INV_OK
+    return out
+
+
+def bench_prefill(inv, torch, device, cfg, w, T=8192, chunk=512):
+    """One layer over a T-token prompt of one sequence: prefill_layer one shot
+    and in chunks (each attention split is loaded once per chunk)."""
+    from invariant_numerics_b200 import synth
+    max_len = (T + 63) // 64 * 64
+    pcfg = inv.LayerConfig(hidden=cfg.hidden, n_heads=cfg.n_heads, n_kv_heads=cfg.n_kv_heads, ffn=cfg.ffn,
+                           max_pos=cfg.max_pos)
+    if pcfg.max_pos < max_len:
+        return {"skipped": f"rotary tables cover {pcfg.max_pos} positions < {T}"}
+    x = torch.from_numpy(synth.normal((T, cfg.hidden), seed=77)).to(device)
+    out = {}
+    for name, step in (("one_shot", T), (f"chunk{chunk}", chunk)):
+        cache = inv.KVCache(n_slots=1, n_kv_heads=cfg.n_kv_heads, max_len=max_len, device=device)
+        y = torch.empty_like(x)
+
+        def run():
+            for a in range(0, T, step):
+                inv.prefill_layer(pcfg, w, cache, x[a:a + step], 0, a, out=y[a:a + step])
+        run()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run()
+        e1.record()
+        e1.synchronize()
+        ms = e0.elapsed_time(e1)
+        out[name] = {"ms": round(ms, 3), "tokens_per_s": round(T / (ms * 1e-3), 1)}
+    assert inv.inv_get_device_status() == inv.INV_OK
+    out["tokens"] = T
     return out
 
 
