@@ -62,7 +62,7 @@ typedef enum {
 /* Fixed algorithm constants (part of the numerics; not tunable). */
 #define INV_KV_SPLIT 256        /* keys per attention split, at absolute positions 256*s */
 #define INV_GEMM_BM 128         /* rows per compensated-GEMM tile */
-#define INV_GEMM_BN 64          /* output columns per tile (= packed panel width) */
+#define INV_GEMM_BN 128         /* output columns per tile (= packed panel width) */
 #define INV_GEMM_BK 64          /* K per pipeline stage; K must be a multiple of it */
 #define INV_GEMM_KGROUP 256     /* K per tensor-memory accumulation group */
 #define INV_HEAD_DIM 128        /* the only supported attention head size */
@@ -129,11 +129,11 @@ INV_API int heal_split(const float* x, int64_t rows, int64_t cols, int64_t ld_x,
  * weight matrix W fp32 [K][N] (row-major, y = x W).  For every output column
  * n a static exponent e_n makes max_k |W[k][n]| 2^e_n fall in [2^14, 2^15)
  * (0 for an all-zero column; clamped to [-120, 120]); then W 2^e_n is split
- * like heal_split.  The packed image is binary16 [N/64][2][64][K]: panel j
- * holds the hi rows of its 64 columns, then their lo rows, each contiguous in
+ * like heal_split.  The packed image is binary16 [N/128][2][128][K]: panel j
+ * holds the hi rows of its 128 columns, then their lo rows, each contiguous in
  * K.  Needs heal_packed_weight_bytes(K, N) bytes at `packed`; col_exp is int8 [N].
  * Errors: INV_ERR_INVALID_ARG; INV_ERR_UNSUPPORTED_SHAPE unless K % 64 == 0
- * and N % 64 == 0; INV_ERR_WORKSPACE if packed_bytes is too small.
+ * and N % 128 == 0; INV_ERR_WORKSPACE if packed_bytes is too small.
  * ------------------------------------------------------------------------ */
 INV_API size_t heal_packed_weight_bytes(int K, int N);
 INV_API int heal_pack_weight(const float* W, int K, int N, uint16_t* packed, size_t packed_bytes,
@@ -155,7 +155,7 @@ INV_API int heal_pack_weight(const float* W, int K, int N, uint16_t* packed, siz
  *   y          : fp32 [M][ld_y].   residual : fp32 [M][ld_r] or NULL.
  *                y may alias residual exactly (same pointer and ld).
  * Errors: INV_ERR_INVALID_ARG; INV_ERR_UNSUPPORTED_SHAPE unless K % 64 == 0,
- * N % 64 == 0, K >= 64; M == 0 is a no-op.  Device: INV_ERR_TIMEOUT.
+ * N % 128 == 0, K >= 64; M == 0 is a no-op.  Device: INV_ERR_TIMEOUT.
  * ------------------------------------------------------------------------ */
 INV_API int comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
               const uint16_t* w_packed, const int8_t* col_exp, int N,
@@ -282,7 +282,7 @@ INV_API int rmsnorm_bi(const float* x, const float* gamma, int64_t rows, int hid
  * Errors: as the component calls; INV_ERR_WORKSPACE.
  * ------------------------------------------------------------------------ */
 typedef struct {
-  int hidden;          /* H, multiple of 64 */
+  int hidden;          /* H, multiple of 128 */
   int n_heads;         /* Hq */
   int n_kv_heads;      /* Hkv; Hq / Hkv in {1, 2, 4} */
   int head_dim;        /* must be 128 */

@@ -5,23 +5,26 @@
 // With a = a_hi + 2^-11 a_lo and w 2^e = w_hi + 2^-11 w_lo (binary16 pairs):
 //   y = ( sum a_hi w_hi  +  2^-11 sum (a_hi w_lo + a_lo w_hi) ) 2^-e   [+ residual]
 // Batch invariance ("Defeating Nondeterminism" summary, table row MatMul):
-// ONE tile (128 x 64), ONE K order, no split-K, whatever M is.
+// ONE tile (128 x 128), ONE K order, no split-K, whatever M is.
 //
-// Per 128 x 64 output tile and per 64-wide K block, the MMA thread issues for
+// Per 128 x 128 output tile and per 64-wide K block, the MMA thread issues for
 // each 16-wide K step:
-//   MMA1  D[0:128)  (+)= A_hi * [W_hi ; W_lo]^T   (N = 128: columns 0..63 "hh",
-//                                                  64..127 the first cross term)
-//   MMA2  D[64:128) += A_lo * W_hi^T              (N = 64: second cross term)
-// Accumulation runs in tensor memory over a group of 256 K values (4 blocks),
-// then the epilogue warps read the group (tcgen05.ld) and add it to fp32
-// registers with round-to-nearest adds, groups in ascending K.  Restarting
-// the tensor-memory accumulator every 256 K bounds the error of the tensor
-// core's internal accumulation, whatever K is.  Two group buffers (2 x 128
-// TMEM columns) let the MMAs of group g+1 overlap the drain of group g.
+//   MMA1  D[0:256)   (+)= A_hi * [W_hi ; W_lo]^T  (N = 256: columns 0..127 "hh",
+//                                                  128..255 the first cross term)
+//   MMA2  D[128:256) += A_lo * W_hi^T              (N = 128: second cross term)
+// The tile is 128 wide because a tcgen05.mma costs the issuing thread about the
+// same whatever its N up to 256: with N = 256 + 128 per K step the tensor pipe,
+// not the issue loop, sets the pace.  Accumulation runs in tensor memory over a
+// group of 256 K values (4 blocks), then the epilogue warps read the group
+// (tcgen05.ld) and add it to fp32 registers with round-to-nearest adds, groups
+// in ascending K.  Restarting the tensor-memory accumulator every 256 K bounds
+// the error of the tensor core's internal accumulation, whatever K is.  Two
+// group buffers (2 x 256 TMEM columns, all of tensor memory) let the MMAs of
+// group g+1 overlap the drain of group g.
 //
-// Warp roles (320 threads): warp 0 = TMA producer (4 stages of A_hi, A_lo and
-// the weight panel), warp 1 = TMEM allocator + MMA issuer, warps 2..9 =
-// epilogue (warp w reads TMEM lanes 32*(w%4).., the column half (w-2)/4).
+// Warp roles (320 threads): warp 0 = TMA producer (3 stages of A_hi, A_lo and
+// the 256-row weight panel), warp 1 = TMEM allocator + MMA issuer, warps 2..9 =
+// epilogue (warp w reads TMEM lanes 32*(w%4).., output columns 64*((w-2)/4)..).
 // For M < 128 only round_up(M, 8) A rows are loaded (the MMA's other rows hold
 // stale data and produce output rows that are never stored).  Persistent grid over tiles ordered
 // N-panel-major so a wave of CTAs shares weight panels and A stays in L2.
@@ -31,19 +34,21 @@
 namespace {
 
 constexpr int BM = INV_GEMM_BM;            // 128
-constexpr int BN = INV_GEMM_BN;            // 64
+constexpr int BN = INV_GEMM_BN;            // 128
 constexpr int BK = INV_GEMM_BK;            // 64
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
 constexpr int GROUP_KB = INV_GEMM_KGROUP / BK;  // 4
 constexpr int A_BYTES = BM * BK * 2;       // 16 KB
-constexpr int W_BYTES = 2 * BN * BK * 2;   // 16 KB: 64 hi rows then 64 lo rows
+constexpr int W_BYTES = 2 * BN * BK * 2;   // 32 KB: 128 hi rows then 128 lo rows
 constexpr int STAGE_BYTES = 2 * A_BYTES + W_BYTES;
 constexpr int ACC_COLS = 2 * BN;           // hh | cross
 constexpr int TMEM_COLS = 2 * ACC_COLS;    // two group buffers
 constexpr int EPI_WARPS = 8;
+constexpr int EPI_COLS = BN / 2;           // output columns per epilogue thread
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
+constexpr uint32_t IDESC_N256 = inv::idesc_f16_f32(128, 256);
 constexpr uint32_t IDESC_N128 = inv::idesc_f16_f32(128, 128);
-constexpr uint32_t IDESC_N64 = inv::idesc_f16_f32(128, 64);
+static_assert(TMEM_COLS <= 512, "tensor memory holds 512 columns");
 
 struct __align__(1024) GemmSmem {
   uint8_t stage[STAGES][STAGE_BYTES];
@@ -143,8 +148,8 @@ __global__ void __launch_bounds__(THREADS, 1)
               const uint64_t ahi = inv::sw128_kmajor_desc(base + kk * 32);
               const uint64_t alo = inv::sw128_kmajor_desc(base + A_BYTES + kk * 32);
               const uint64_t bw = inv::sw128_kmajor_desc(base + 2 * A_BYTES + kk * 32);
-              inv::umma_f16(d, ahi, bw, IDESC_N128, (kb > kb0 || kk > 0) ? 1u : 0u);
-              inv::umma_f16(d + BN, alo, bw, IDESC_N64, 1u);
+              inv::umma_f16(d, ahi, bw, IDESC_N256, (kb > kb0 || kk > 0) ? 1u : 0u);
+              inv::umma_f16(d + BN, alo, bw, IDESC_N128, 1u);
             }
             inv::umma_commit(&sm.empty[stage]);
             if (++stage == STAGES) {
@@ -163,13 +168,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue --
     const int quarter = warp & 3;          // TMEM lanes 32*quarter .. +31
-    const int half = (warp - 2) >> 2;      // output columns 32*half .. +31
+    const int half = (warp - 2) >> 2;      // output columns EPI_COLS*half .. +EPI_COLS-1
     uint32_t g = 0;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
       const int nt = tile / tiles_m, mt = tile - nt * tiles_m;
-      float acc_h[32], acc_x[32];
+      float acc_h[EPI_COLS], acc_x[EPI_COLS];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) acc_h[i] = acc_x[i] = 0.0f;
+      for (int i = 0; i < EPI_COLS; ++i) acc_h[i] = acc_x[i] = 0.0f;
       for (int grp = 0; grp < ngroups; ++grp, ++g) {
         const uint32_t buf = g & 1u, tph = (g >> 1) & 1u;
         int okw = 1;
@@ -177,64 +182,69 @@ __global__ void __launch_bounds__(THREADS, 1)
         okw = __shfl_sync(0xffffffffu, okw, 0);  // keep the warp converged for tcgen05.ld
         if (!okw) goto epi_done;
         inv::tc_fence_after();
-        const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * ACC_COLS + half * 32;
-        uint32_t rh[32], rx[32];
-        inv::tmem_ld_32x32(ta, rh);
-        inv::tmem_ld_32x32(ta + BN, rx);
-        inv::tmem_wait_ld();
+        const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * ACC_COLS + half * EPI_COLS;
+#pragma unroll
+        for (int c = 0; c < EPI_COLS; c += 16) {
+          uint32_t rh[16], rx[16];
+          inv::tmem_ld_32x16(ta + c, rh);
+          inv::tmem_ld_32x16(ta + BN + c, rx);
+          inv::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            acc_h[c + i] = __fadd_rn(acc_h[c + i], __uint_as_float(rh[i]));
+            acc_x[c + i] = __fadd_rn(acc_x[c + i], __uint_as_float(rx[i]));
+          }
+        }
         inv::tc_fence_before();
         __syncwarp();
         if (lane == 0) inv::mbar_arrive(&sm.tempty[buf]);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          acc_h[i] = __fadd_rn(acc_h[i], __uint_as_float(rh[i]));
-          acc_x[i] = __fadd_rn(acc_x[i], __uint_as_float(rx[i]));
-        }
       }
       {
         const int row = mt * BM + quarter * 32 + lane;
+        const int col0 = nt * BN + half * EPI_COLS;
         if (row < M && gate_hi != nullptr) {
-          // Fused SwiGLU: this thread's 32 packed columns are 16 gate columns
-          // then the 16 matching up columns of outputs f0 .. f0+15.
-          const int col0 = nt * BN + half * 32;
-          const int f0 = nt * (BN / 2) + half * 16;
-          float v[32];
+          // Fused SwiGLU: each 32 packed columns are 16 gate columns then the
+          // 16 matching up columns of outputs f0 .. f0+15, f0 = column / 2.
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const char4 e4 = *reinterpret_cast<const char4*>(col_exp + col0 + i);
-            const int ev[4] = {e4.x, e4.y, e4.z, e4.w};
+          for (int c = 0; c < EPI_COLS; c += 32) {
+            const int f0 = (col0 + c) / 2;
+            float v[32];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float t = __fadd_rn(acc_h[i + j], __fmul_rn(acc_x[i + j], 0x1p-11f));
-              v[i + j] = __fmul_rn(t, inv::pow2f(-ev[j]));
+            for (int i = 0; i < 32; i += 4) {
+              const char4 e4 = *reinterpret_cast<const char4*>(col_exp + col0 + c + i);
+              const int ev[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const float t = __fadd_rn(acc_h[c + i + j], __fmul_rn(acc_x[c + i + j], 0x1p-11f));
+                v[i + j] = __fmul_rn(t, inv::pow2f(-ev[j]));
+              }
             }
-          }
-          uint32_t hw[8], lw[8];
-          bool bad = false;
+            uint32_t hw[8], lw[8];
+            bool bad = false;
 #pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            __half h0, l0, h1, l1;
-            const float a0 = __fmul_rn(__fdiv_rn(v[i], __fadd_rn(1.0f, expf(-v[i]))), v[16 + i]);
-            const float a1 = __fmul_rn(__fdiv_rn(v[i + 1], __fadd_rn(1.0f, expf(-v[i + 1]))), v[17 + i]);
-            bad |= inv::f16_overflow(a0) | inv::f16_overflow(a1);
-            inv::split_hi_lo(a0, h0, l0);
-            inv::split_hi_lo(a1, h1, l1);
-            hw[i / 2] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
-            lw[i / 2] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
+            for (int i = 0; i < 16; i += 2) {
+              __half h0, l0, h1, l1;
+              const float a0 = __fmul_rn(__fdiv_rn(v[i], __fadd_rn(1.0f, expf(-v[i]))), v[16 + i]);
+              const float a1 = __fmul_rn(__fdiv_rn(v[i + 1], __fadd_rn(1.0f, expf(-v[i + 1]))), v[17 + i]);
+              bad |= inv::f16_overflow(a0) | inv::f16_overflow(a1);
+              inv::split_hi_lo(a0, h0, l0);
+              inv::split_hi_lo(a1, h1, l1);
+              hw[i / 2] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
+              lw[i / 2] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
+            }
+            if (bad) inv::record_status(status, INV_ERR_RANGE);
+            uint4* gh = reinterpret_cast<uint4*>(gate_hi + (int64_t)row * ld_g + f0);
+            uint4* gl = reinterpret_cast<uint4*>(gate_lo + (int64_t)row * ld_g + f0);
+            gh[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            gh[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+            gl[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            gl[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
           }
-          if (bad) inv::record_status(status, INV_ERR_RANGE);
-          uint4* gh = reinterpret_cast<uint4*>(gate_hi + (int64_t)row * ld_g + f0);
-          uint4* gl = reinterpret_cast<uint4*>(gate_lo + (int64_t)row * ld_g + f0);
-          gh[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          gh[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
-          gl[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-          gl[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
         } else if (row < M) {
-          const int col0 = nt * BN + half * 32;
           float* yr = y + (int64_t)row * ld_y + col0;
           const float* rr = residual ? residual + (int64_t)row * ld_r + col0 : nullptr;
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
+          for (int i = 0; i < EPI_COLS; i += 4) {
             const char4 e4 = *reinterpret_cast<const char4*>(col_exp + col0 + i);
             const int ev[4] = {e4.x, e4.y, e4.z, e4.w};
             float o[4];

@@ -63,7 +63,7 @@ int validate(const inv_layer_config* cfg, const inv_kv_cache* cache) {
   if (cfg->head_dim != INV_HEAD_DIM || cache->head_dim != INV_HEAD_DIM) return INV_ERR_UNSUPPORTED_SHAPE;
   if (cfg->hidden <= 0 || cfg->ffn <= 0 || cfg->n_heads <= 0 || cfg->n_kv_heads <= 0 || cfg->max_pos <= 0)
     return INV_ERR_INVALID_ARG;
-  if (cfg->hidden % 64 != 0 || cfg->ffn % 64 != 0) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (cfg->hidden % INV_GEMM_BN != 0 || cfg->ffn % 64 != 0) return INV_ERR_UNSUPPORTED_SHAPE;
   if (cfg->n_heads % cfg->n_kv_heads != 0) return INV_ERR_UNSUPPORTED_SHAPE;
   const int G = cfg->n_heads / cfg->n_kv_heads;
   if (G != 1 && G != 2 && G != 4) return INV_ERR_UNSUPPORTED_SHAPE;

@@ -83,23 +83,25 @@ __global__ void col_exp_kernel(const float* __restrict__ W, int K, int N, int8_t
   e_out[n] = (int8_t)e;
 }
 
-// Packed image [N/64][2][64][K]; a block transposes a 64(k) x 64(n) tile.
+// Packed image [N/128][2][128][K]; a block transposes a 64(k) x 64(n) tile.
 __global__ void pack_kernel(const float* __restrict__ W, int K, int N, const int8_t* __restrict__ e,
                             __half* __restrict__ P) {
+  constexpr int PW = INV_GEMM_BN;    // panel width
   __shared__ float tile[64][65];
-  const int j = blockIdx.x;          // panel (64 columns)
+  const int n0 = blockIdx.x * 64;    // 64 columns, inside one panel
   const int k0 = blockIdx.y * 64;
   const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 256 threads: 64 x 4
-  for (int kk = ty; kk < 64; kk += 4) tile[kk][tx] = W[(int64_t)(k0 + kk) * N + j * 64 + tx];
+  for (int kk = ty; kk < 64; kk += 4) tile[kk][tx] = W[(int64_t)(k0 + kk) * N + n0 + tx];
   __syncthreads();
   for (int r = ty; r < 64; r += 4) {
-    const int n = j * 64 + r;
+    const int n = n0 + r;
+    const int j = n / PW, rr = n % PW;
     const float s = inv::pow2f(e[n]);
     const float v = __fmul_rn(tile[tx][r], s);  // exact power-of-two scaling
     __half h, l;
     split_hi_lo(v, h, l);
-    P[(((int64_t)j * 2 + 0) * 64 + r) * K + k0 + tx] = h;
-    P[(((int64_t)j * 2 + 1) * 64 + r) * K + k0 + tx] = l;
+    P[(((int64_t)j * 2 + 0) * PW + rr) * K + k0 + tx] = h;
+    P[(((int64_t)j * 2 + 1) * PW + rr) * K + k0 + tx] = l;
   }
 }
 
@@ -477,7 +479,7 @@ size_t heal_packed_weight_bytes(int K, int N) {
 int heal_pack_weight(const float* W, int K, int N, uint16_t* packed, size_t packed_bytes, int8_t* col_exp,
                      inv_stream stream) {
   if (!W || !packed || !col_exp || K <= 0 || N <= 0) return INV_ERR_INVALID_ARG;
-  if (K % 64 != 0 || N % 64 != 0) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (K % 64 != 0 || N % INV_GEMM_BN != 0) return INV_ERR_UNSUPPORTED_SHAPE;
   if (packed_bytes < heal_packed_weight_bytes(K, N)) return INV_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   col_exp_kernel<<<(N + 255) / 256, 256, 0, s>>>(W, K, N, col_exp);

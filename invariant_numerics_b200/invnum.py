@@ -163,10 +163,10 @@ def heal_split(x, hi=None, lo=None, stream=None):
 
 
 def heal_pack_weight(W, stream=None):
-    """fp32 W [K, N] (y = x W) -> (packed binary16 [N/64, 2, 64, K], col_exp int8 [N])."""
+    """fp32 W [K, N] (y = x W) -> (packed binary16 [N/128, 2, 128, K], col_exp int8 [N])."""
     _need(W, torch.float32, "W")
     K, N = W.shape
-    packed = torch.empty((N // 64, 2, 64, K), dtype=torch.float16, device=W.device)
+    packed = torch.empty((N // 128, 2, 128, K), dtype=torch.float16, device=W.device)
     col_exp = torch.empty((N,), dtype=torch.int8, device=W.device)
     nbytes = lib.heal_packed_weight_bytes(K, N)
     _check("heal_pack_weight", lib.heal_pack_weight(_ptr(W), K, N, _ptr(packed), nbytes, _ptr(col_exp),

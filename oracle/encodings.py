@@ -102,7 +102,7 @@ def f16_bits_to_f64(bits) -> np.ndarray:
 # most 2^-22 |x| whenever 2^-14 <= |x 2^e| < 65520.
 
 LO_SCALE_LOG2 = 11
-PACK_BN = 64  # output columns per packed weight panel (layout constant)
+PACK_BN = 128  # output columns per packed weight panel (layout constant)
 
 
 def heal_split(x, e=0):
@@ -144,9 +144,9 @@ def heal_pack_weight(W):
     """Packed weight image and column exponents for the compensated GEMM.
 
     W is fp32 [K, N] (y = x W), N a multiple of PACK_BN.  The image is binary16
-    bit patterns laid out [N/64][2][64][K]: panel j holds, for its 64 output
-    columns n = 64 j + r, first the hi rows then the lo rows, each row
-    contiguous along K.  Returns (packed uint16 [N/64, 2, 64, K], e int8 [N]).
+    bit patterns laid out [N/128][2][128][K]: panel j holds, for its 128 output
+    columns n = 128 j + r, first the hi rows then the lo rows, each row
+    contiguous along K.  Returns (packed uint16 [N/128, 2, 128, K], e int8 [N]).
     """
     W = np.asarray(W, dtype=np.float32)
     K, N = W.shape

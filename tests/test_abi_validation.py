@@ -46,7 +46,8 @@ def test_split_pack_norm_quant_validation(inv, L):
     assert L.heal_split(P, -1, 8, 8, P, P, 8, None) == INVALID
     assert L.heal_split(P, 4, 8, 4, P, P, 8, None) == INVALID
     assert L.heal_pack_weight(P, 100, 64, P, 10 ** 9, P, None) == UNSUPPORTED
-    assert L.heal_pack_weight(P, 64, 64, P, 10, P, None) == WORKSPACE
+    assert L.heal_pack_weight(P, 64, 64, P, 10 ** 9, P, None) == UNSUPPORTED       # N % 128
+    assert L.heal_pack_weight(P, 64, 128, P, 10, P, None) == WORKSPACE
     assert L.rmsnorm_bi(P, P, 4, 6, 1e-6, P, None, None, None) == UNSUPPORTED
     assert L.rmsnorm_bi(P, P, 0, 64, 1e-6, P, None, None, None) == OK
     assert L.rmsnorm_bi(P, P, 4, 64, 1e-6, P, P, None, None) == INVALID          # hi without lo

@@ -50,11 +50,11 @@ def test_heal_split_range_error(inv):
 
 
 def test_pack_weight_bit_exact(inv):
-    for K, N, std in ((512, 512, 0.02), (1024, 192, 3.0), (64, 64, 1e-6)):
+    for K, N, std in ((512, 512, 0.02), (1024, 384, 3.0), (64, 128, 1e-6)):
         W = synth.normal((K, N), seed=K + N, std=std)
         W[0, 0] = 0.0
-        if N > 64:
-            W[:, 64:128] = 0.0  # an all-zero panel
+        if N > 128:
+            W[:, 128:256] = 0.0  # an all-zero panel
         P, e = inv.heal_pack_weight(dev(W))
         P_want, e_want = enc.heal_pack_weight(W)
         assert np.array_equal(host(e), e_want)
@@ -210,8 +210,8 @@ def test_comp_gemm_ragged_and_residual(inv):
 
 def test_comp_gemm_rejects_bad_shapes(inv):
     hi = torch.zeros((4, 100), dtype=torch.float16, device="cuda")
-    P = torch.zeros((1, 2, 64, 100), dtype=torch.float16, device="cuda")
-    e = torch.zeros((64,), dtype=torch.int8, device="cuda")
+    P = torch.zeros((1, 2, 128, 100), dtype=torch.float16, device="cuda")
+    e = torch.zeros((128,), dtype=torch.int8, device="cuda")
     with pytest.raises(inv.InvError) as ei:
         inv.comp_gemm(hi, hi, P, e)       # K % 64 != 0
     assert ei.value.code == inv.INV_ERR_UNSUPPORTED_SHAPE

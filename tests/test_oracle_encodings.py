@@ -140,24 +140,24 @@ def test_column_exponents_closed_form():
 
 
 def test_pack_weight_layout_and_values():
-    K, N = 64, 128
+    K, N = 64, 256
     # W[k, n] built from small integers and a per-column power of two so the
     # scaled values are exact binary16 numbers (lo == 0) with a known position.
     k = np.arange(K)[:, None]
     n = np.arange(N)[None, :]
     W = ((k + 1) * 3 + (n % 7)).astype(np.float32) * np.float32(2.0**-6)
     P, e = enc.heal_pack_weight(W)
-    assert P.shape == (N // 64, 2, 64, K) and P.dtype == np.uint16
-    for j in range(N // 64):
-        for r in (0, 5, 63):
-            col = 64 * j + r
+    assert P.shape == (N // 128, 2, 128, K) and P.dtype == np.uint16
+    for j in range(N // 128):
+        for r in (0, 5, 64, 127):
+            col = 128 * j + r
             hv = enc.f16_bits_to_f64(P[j, 0, r, :])
             lv = enc.f16_bits_to_f64(P[j, 1, r, :])
             assert (hv == W[:, col].astype(np.float64) * 2.0**int(e[col])).all()
             assert (lv == 0).all()
     # a generic matrix reconstructs within 2^-22 relative on normal elements
     g = np.random.Generator(np.random.PCG64(3))
-    W2 = (g.standard_normal((128, 64)) * 0.02).astype(np.float32)
+    W2 = (g.standard_normal((128, 128)) * 0.02).astype(np.float32)
     P2, e2 = enc.heal_pack_weight(W2)
     rec = enc.heal_reconstruct(P2[0, 0].T, P2[0, 1].T, e2[None, :].astype(np.int64))
     normal = np.abs(W2) * 2.0**e2[None, :].astype(np.float64) >= 2.0**-14
