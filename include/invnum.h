@@ -203,7 +203,7 @@ INV_API int kv_quant_int16(const float* x, int T, int64_t ld_x, const int32_t* s
  * hi/lo split of q, its own max, exp-sum and value sum; the splits are then
  * folded in ascending s.  Nothing depends on other rows or on len beyond the
  * row's own split count.
- *   q        : fp32 [B][n_heads][128].
+ *   q        : fp32 [B][n_heads][128], 16-byte aligned.
  *   len      : int32 [B], 1 <= len[b] <= cache->max_len.
  *   max_len_bound : host upper bound on every len[b] (<= 0: cache->max_len);
  *                   only sizes the launch grid.

@@ -46,6 +46,7 @@ struct RowScratch {
 
 struct __align__(1024) DecodeSmem {
   uint8_t codes[CODE_BYTES];   // K codes, then V codes, then the warp exchange of O
+  float qs[4 * 128];           // q of the row's G query heads (bulk copy with K)
   float ks[SPLIT];
   float vs[SPLIT];
   RowScratch rs;
@@ -341,8 +342,11 @@ __global__ void __launch_bounds__(THREADS, 3)
     inv::fence_mbar_init();
   }
   __syncthreads();
+  const int64_t obase = (int64_t)b * Hq + (int64_t)h * G;
   if (tid == 0) {
-    inv::mbar_arrive_expect_tx(&sm.bar_k, nbox * 2 * BOX_BYTES);
+    // q travels with K, so the scores start as soon as the codes land
+    inv::mbar_arrive_expect_tx(&sm.bar_k, nbox * 2 * BOX_BYTES + G * 128 * 4);
+    inv::bulk_load(sm.qs, q + obase * 128, (uint32_t)(G * 128 * 4), &sm.bar_k);
     for (int bx = 0; bx < nbox; ++bx) {
       inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES, &tm_k, &sm.bar_k, 0, row0 + 64 * bx);
       inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES + BOX_BYTES, &tm_k, &sm.bar_k, 64, row0 + 64 * bx);
@@ -359,9 +363,8 @@ __global__ void __launch_bounds__(THREADS, 3)
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 
   bool v_issued = false;
-  const int64_t obase = (int64_t)b * Hq + (int64_t)h * G;
   split_row<false>(
-      q + obase * 128, G, n, cbase, cbase, sm.ks, sm.vs, sm.rs, reinterpret_cast<float*>(sm.codes), sigma,
+      sm.qs, G, n, cbase, cbase, sm.ks, sm.vs, sm.rs, reinterpret_cast<float*>(sm.codes), sigma,
       part_o + (obase * S_max + s) * 128, part_ml + obase * S_max + s, (int64_t)S_max * 128, (int64_t)S_max, ok,
       status,
       [&]() {  // every warp is done with K: bring V into the same buffer
@@ -630,7 +633,8 @@ int attn_decode_fixedsplit(const float* q, int B, int n_heads, const inv_kv_cach
   if (!q || !slot || !len || !out || !cache->k || !cache->v || !cache->k_scale || !cache->v_scale || !workspace)
     return INV_ERR_INVALID_ARG;
   if ((out_hi == nullptr) != (out_lo == nullptr)) return INV_ERR_INVALID_ARG;
-  if (!inv::aligned16(cache->k) || !inv::aligned16(cache->v) || !inv::aligned16(out) || !inv::aligned16(workspace))
+  if (!inv::aligned16(q) || !inv::aligned16(cache->k) || !inv::aligned16(cache->v) || !inv::aligned16(out) ||
+      !inv::aligned16(workspace))
     return INV_ERR_INVALID_ARG;
   if (out_hi && ((reinterpret_cast<uintptr_t>(out_hi) | reinterpret_cast<uintptr_t>(out_lo)) & 7u))
     return INV_ERR_INVALID_ARG;

@@ -65,7 +65,8 @@ extern "C" int attn_decode_fixedsplit_noalloc(const float* q, int B, int n_heads
   if (!q || !slot || !len || !out || !cache->k || !cache->v || !cache->k_scale || !cache->v_scale)
     return INV_ERR_INVALID_ARG;
   if ((out_hi == nullptr) != (out_lo == nullptr)) return INV_ERR_INVALID_ARG;
-  if (!inv::aligned16(cache->k) || !inv::aligned16(cache->v) || !inv::aligned16(out)) return INV_ERR_INVALID_ARG;
+  if (!inv::aligned16(q) || !inv::aligned16(cache->k) || !inv::aligned16(cache->v) || !inv::aligned16(out))
+    return INV_ERR_INVALID_ARG;
   if (out_hi && ((reinterpret_cast<uintptr_t>(out_hi) | reinterpret_cast<uintptr_t>(out_lo)) & 7u))
     return INV_ERR_INVALID_ARG;
   const int mlb =

@@ -67,6 +67,7 @@ def test_attention_validation(inv, L):
     assert a(P, 4, 32, C.byref(c), P, P, 256, 256, 0.1, P, None, None, P, 16, None) == WORKSPACE
     assert a(P, 0, 32, C.byref(c), P, P, 256, 256, 0.1, P, None, None, P, 16, None) == OK
     assert a(P, 4, 32, C.byref(c), P, P, 256, 256, 0.1, P, P, None, P, 10 ** 9, None) == INVALID  # hi w/o lo
+    assert a(MISALIGNED, 4, 32, C.byref(c), P, P, 256, 256, 0.1, P, None, None, P, 10 ** 9, None) == INVALID  # q
     need = L.attn_decode_workspace_size(4, 32, 256)
     assert need == 4 * 32 * 1 * 520
     c_big = cache(inv, max_len=8192)
