@@ -50,7 +50,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # 2048, from the ncu capture in profiles/attn_split_B32_kv2048.md (B = 32:
 # 273.22 MB read + 6.52 MB written), scaled by rows.  Set to None whenever the
 # kernel changes until it is captured again.
-ATTN_SPLIT_DRAM_BYTES_PER_ROW_KV2048 = (273.221632e6 + 7.541760e6) / 32
+ATTN_SPLIT_DRAM_BYTES_PER_ROW_KV2048 = (273.218560e6 + 6.921984e6) / 32
 
 
 def load_peaks():

@@ -50,7 +50,7 @@ struct __align__(1024) DecodeSmem {
   float ks[SPLIT];
   float vs[SPLIT];
   RowScratch rs;
-  uint64_t bar_k, bar_v;
+  uint64_t bar_k, bar_v[4];    // V: one barrier per warp (its 64 keys)
   int abort;
 };
 constexpr size_t kDecodeSmem = sizeof(DecodeSmem) + 1024;
@@ -123,8 +123,10 @@ __device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
 //   ks/vs : shared scales (zero beyond the keys that were loaded).
 //   xo   : shared [4 warps][4 heads][128] exchange buffer (may alias the codes
 //          in the decode kernel: it is written only after the last V read).
-//   issue_v / wait_v : hooks around the first V access (decode kernel: load V
-//          into the K buffer once every warp is done with K).
+//   issue_v / wait_v : hooks around the first V access.  issue_v runs in every
+//          thread once its warp has finished reading K (a warp reads and later
+//          overwrites only the codes of its own 64 keys); the decode kernel
+//          loads that warp's V codes into the warp's K slot there.
 //   out_o/out_ml : this row's partials for head 0 of the group, split s.
 template <bool kReuse, class IssueV, class WaitV>
 __device__ __forceinline__ void split_row(const float* __restrict__ qrow, int G, int n, uint32_t kbase,
@@ -194,9 +196,10 @@ __device__ __forceinline__ void split_row(const float* __restrict__ qrow, int G,
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
   if (g == 0) rs.red_m[warp][c] = mx;
-  inv::fence_proxy_async_smem();  // K reads (generic proxy) before any TMA overwrite (async proxy)
-  __syncthreads();
+  inv::fence_proxy_async_smem();  // this warp's K reads (generic proxy) before the TMA overwrite (async proxy)
+  __syncwarp();
   issue_v();
+  __syncthreads();
 
   // ---------------------------------------------------------------- softmax --
   const float M = fmaxf(fmaxf(rs.red_m[0][c], rs.red_m[1][c]), fmaxf(rs.red_m[2][c], rs.red_m[3][c]));
@@ -337,7 +340,7 @@ __global__ void __launch_bounds__(THREADS, 3)
 
   if (tid == 0) {
     inv::mbar_init(&sm.bar_k, 1);
-    inv::mbar_init(&sm.bar_v, 1);
+    for (int w = 0; w < 4; ++w) inv::mbar_init(&sm.bar_v[w], 1);
     sm.abort = 0;
     inv::fence_mbar_init();
   }
@@ -367,26 +370,24 @@ __global__ void __launch_bounds__(THREADS, 3)
       sm.qs, G, n, cbase, cbase, sm.ks, sm.vs, sm.rs, reinterpret_cast<float*>(sm.codes), sigma,
       part_o + (obase * S_max + s) * 128, part_ml + obase * S_max + s, (int64_t)S_max * 128, (int64_t)S_max, ok,
       status,
-      [&]() {  // every warp is done with K: bring V into the same buffer
-        if (tid == 0 && ok) {
+      [&]() {  // this warp is done with its K codes: bring its V codes into the same slot
+        const int warp = tid >> 5;
+        if (lane == 0 && ok && warp < nbox) {
           v_issued = true;
-          inv::mbar_arrive_expect_tx(&sm.bar_v, nbox * 2 * BOX_BYTES);
-          for (int bx = 0; bx < nbox; ++bx) {
-            inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES, &tm_v, &sm.bar_v, 0, row0 + 64 * bx);
-            inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES + BOX_BYTES, &tm_v, &sm.bar_v, 64, row0 + 64 * bx);
-          }
+          inv::mbar_arrive_expect_tx(&sm.bar_v[warp], 2 * BOX_BYTES);
+          inv::tma_load_2d(sm.codes + warp * 2 * BOX_BYTES, &tm_v, &sm.bar_v[warp], 0, row0 + 64 * warp);
+          inv::tma_load_2d(sm.codes + warp * 2 * BOX_BYTES + BOX_BYTES, &tm_v, &sm.bar_v[warp], 64, row0 + 64 * warp);
         }
       },
       [&](bool okv) {
-        if (lane == 0 && okv) okv = inv::mbar_wait(&sm.bar_v, 0, wait_ns, &sm.abort, status);
+        const int warp = tid >> 5;
+        if (lane == 0 && okv && warp < nbox) okv = inv::mbar_wait(&sm.bar_v[warp], 0, wait_ns, &sm.abort, status);
         return __shfl_sync(0xffffffffu, okv ? 1 : 0, 0) != 0;
       });
   // No copy may still be landing in this CTA's shared memory when it exits
   // (only possible after a timed-out wait; immediate otherwise).
-  if (tid == 0) {
-    inv::mbar_wait(&sm.bar_k, 0, wait_ns, nullptr, status);
-    if (v_issued) inv::mbar_wait(&sm.bar_v, 0, wait_ns, nullptr, status);
-  }
+  if (tid == 0) inv::mbar_wait(&sm.bar_k, 0, wait_ns, nullptr, status);
+  if (lane == 0 && v_issued) inv::mbar_wait(&sm.bar_v[tid >> 5], 0, wait_ns, nullptr, status);
 }
 
 // Prefill: rows r = 0..T-1 of one sequence (slot sl) at positions p0 + r.
