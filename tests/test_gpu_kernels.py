@@ -169,6 +169,22 @@ def test_comp_gemm_invariance_across_row_placement(inv):
     assert status() == inv.INV_OK
 
 
+def test_comp_gemm_invariance_across_column_placement(inv):
+    """A column's bits depend on nothing but its own weights and K order: the
+    same weight columns give the same bits in another panel or another N."""
+    K = 2048
+    A = synth.normal_with_outliers((200, K), seed=15)
+    W = synth.normal((K, 512), seed=16, std=0.02)
+    hi, lo = inv.heal_split(dev(A))
+    P, e = inv.heal_pack_weight(dev(W))
+    full = inv.comp_gemm(hi, lo, P, e)
+    for c0, c1 in ((128, 256), (256, 512), (0, 384)):
+        Ps, es = inv.heal_pack_weight(dev(W[:, c0:c1].copy()))
+        part = inv.comp_gemm(hi, lo, Ps, es)
+        assert torch.equal(part.view(torch.int32), full[:, c0:c1].contiguous().view(torch.int32)), (c0, c1)
+    assert status() == inv.INV_OK
+
+
 @pytest.mark.parametrize("N", [4096, 11008])
 def test_comp_gemm_sweep_parity_and_invariance(inv, N):
     K = 4096
