@@ -47,9 +47,9 @@ H, HQ, HKV, D, F = 4096, 32, 8, 128, 11008
 BATCH, KV_LEN = 128, 2048
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one attn_split launch per decoded row at KV length
-# 2048, from the ncu capture in profiles/attn_split_B32_kv2048.md (B = 32:
-# 273.22 MB read + 6.52 MB written), scaled by rows.  Set to None whenever the
-# kernel changes until it is captured again.
+# 2048, from an ncu capture of the kernel at B = 32 (273.22 MB read + 6.92 MB
+# written), scaled by rows.  Set to None whenever the kernel changes and the
+# capture has not been repeated.
 ATTN_SPLIT_DRAM_BYTES_PER_ROW_KV2048 = (273.218560e6 + 6.921984e6) / 32
 
 
@@ -589,6 +589,45 @@ def run_reference(args, rank, world):
     }), flush=True)
 
 
+def run_gemm_only(args, local):
+    """One compensated GEMM shape, timed with CUDA events (inputs larger than L2
+    are flushed by a 256 MB write before every launch)."""
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    from invariant_numerics_b200 import build as _b
+    _b.build()
+    from invariant_numerics_b200 import invnum as inv
+    from invariant_numerics_b200 import synth
+    M, N, K = args.gemm
+    A = torch.from_numpy(synth.normal_with_outliers((M, K), seed=10)).to(device)
+    W = torch.from_numpy(synth.normal((K, N), seed=11, std=0.02)).to(device)
+    hi, lo = inv.heal_split(A)
+    P, e = inv.heal_pack_weight(W)
+    y = torch.empty((M, N), dtype=torch.float32, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    ts = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        inv.comp_gemm(hi, lo, P, e, out=y)
+        b.record()
+        b.synchronize()
+        if i >= args.warmup:
+            ts.append(a.elapsed_time(b))
+    st = inv.inv_get_device_status()
+    if st != inv.INV_OK:
+        raise RuntimeError(f"device status {inv.status_string(st)}")
+    peaks, kind = load_peaks()
+    us = statistics.median(ts) * 1e3
+    tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+    print(json.dumps({"metric": "comp_gemm useful TFLOP/s", "value": round(tf, 2), "unit": "TFLOP/s",
+                      "config": {"workload": f"comp_gemm M{M} N{N} K{K}"}, "us": round(us, 2),
+                      "frac_of_peak_over_3": round(tf / (peaks["bf16_tflops"] / 3.0), 4),
+                      "steps": args.steps, "warmup": args.warmup}))
+
+
 def main():
     global BATCH, KV_LEN, H, HQ, HKV, F
     ap = argparse.ArgumentParser()
@@ -606,6 +645,8 @@ def main():
     ap.add_argument("--kv", type=int, default=KV_LEN, help="KV length per sequence, multiple of 64")
     ap.add_argument("--oracle-rows", type=int, default=2)
     ap.add_argument("--oracle-seconds", type=float, default=10.0)
+    ap.add_argument("--gemm", type=int, nargs=3, metavar=("M", "N", "K"),
+                    help="time one compensated GEMM shape only (one JSON line; for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -616,7 +657,9 @@ def main():
     rank, world, local = replicas.env_ranks()
     if world > 1 and world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    if args.impl == "reference":
+    if args.gemm:
+        run_gemm_only(args, local)
+    elif args.impl == "reference":
         run_reference(args, rank, world)
     else:
         run_ours(args, rank, world, local)
