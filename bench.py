@@ -440,6 +440,8 @@ def run_ours(args, rank, world, local):
     if not args.no_components and rank == 0:
         result["components"] = bench_components(inv, torch, device, peaks, peak_kind)
         result["components"]["prefill"] = bench_prefill(inv, torch, device, cfg, w)
+        result["components"]["decode_batch_sweep"] = bench_batch_sweep(inv, torch, cfg, w, cache, x, slot, pos,
+                                                                      peaks)
     if not args.no_cpu_baseline and rank == 0 and world == 1:
         v, el, calls = time_oracle(args.oracle_rows, args.oracle_seconds)
         result["cpu_baseline"] = {"value": round(v, 4), "unit": "tokens/s", "cores": cpu_cores_used(),
@@ -552,6 +554,48 @@ def bench_prefill(inv, torch, device, cfg, w, T=8192, chunk=512):
         out[name] = {"ms": round(ms, 3), "tokens_per_s": round(T / (ms * 1e-3), 1)}
     assert inv.inv_get_device_status() == inv.INV_OK
     out["tokens"] = T
+    return out
+
+
+def bench_batch_sweep(inv, torch, cfg, w, cache, x, slot, pos, peaks, batches=(1, 8, 32), reps=300):
+    """The same decode step at smaller batches (the first B sequences of the
+    bench cache), each replayed as a CUDA graph: tokens/s and the fraction of
+    the step's HBM roofline (weights + KV + activations at the measured copy
+    bandwidth)."""
+    out = {}
+    L = KV_LEN
+    for B in batches:
+        if B > x.shape[0]:
+            continue
+        xb, sb, pb = x[:B].clone(), slot[:B].clone(), pos[:B].clone()
+        yb = torch.empty_like(xb)
+        call = inv.DecodeLayerCall(cfg, w, cache, xb, sb, pb, yb)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            call()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call()
+        for _ in range(5):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        e1.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        gemm, attn = layer_bytes(B, L)
+        total = sum(gemm.values()) + attn
+        bound_ms = total / (peaks["hbm_gbs"] * 1e9) * 1e3
+        out[f"B{B}"] = {"ms_per_step": round(ms, 4), "tokens_per_s": round(B / (ms * 1e-3), 1),
+                        "hbm_roofline_frac": round(bound_ms / ms, 4)}
+        del g
+    assert inv.inv_get_device_status() == inv.INV_OK
     return out
 
 

@@ -22,8 +22,9 @@
 // group buffers (2 x 256 TMEM columns, all of tensor memory) let the MMAs of
 // group g+1 overlap the drain of group g.
 //
-// Warp roles (320 threads): warp 0 = TMA producer (3 stages of A_hi, A_lo and
-// the 256-row weight panel), warp 1 = TMEM allocator + MMA issuer, warps 2..9 =
+// Warp roles (320 threads): warp 0 = TMA producer (a 192 KB ring of stages of
+// A_hi, A_lo and the 256-row weight panel: 3 stages at 128 A rows, up to 5 for
+// small M), warp 1 = TMEM allocator + MMA issuer, warps 2..9 =
 // epilogue (warp w reads TMEM lanes 32*(w%4).., output columns 64*((w-2)/4)..).
 // For M < 128 only round_up(M, 8) A rows are loaded (the MMA's other rows hold
 // stale data and produce output rows that are never stored).  Persistent grid over tiles ordered
@@ -36,11 +37,10 @@ namespace {
 constexpr int BM = INV_GEMM_BM;            // 128
 constexpr int BN = INV_GEMM_BN;            // 128
 constexpr int BK = INV_GEMM_BK;            // 64
-constexpr int STAGES = 3;
+constexpr int MAX_STAGES = 8;
+constexpr int RING_BYTES = 3 * (2 * BM * INV_GEMM_BK * 2 + 2 * INV_GEMM_BN * INV_GEMM_BK * 2);  // 192 KB
 constexpr int GROUP_KB = INV_GEMM_KGROUP / BK;  // 4
-constexpr int A_BYTES = BM * BK * 2;       // 16 KB
 constexpr int W_BYTES = 2 * BN * BK * 2;   // 32 KB: 128 hi rows then 128 lo rows
-constexpr int STAGE_BYTES = 2 * A_BYTES + W_BYTES;
 constexpr int ACC_COLS = 2 * BN;           // hh | cross
 constexpr int TMEM_COLS = 2 * ACC_COLS;    // two group buffers
 constexpr int EPI_WARPS = 8;
@@ -51,9 +51,9 @@ constexpr uint32_t IDESC_N128 = inv::idesc_f16_f32(128, 128);
 static_assert(TMEM_COLS <= 512, "tensor memory holds 512 columns");
 
 struct __align__(1024) GemmSmem {
-  uint8_t stage[STAGES][STAGE_BYTES];
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint8_t ring[RING_BYTES];  // n_stages stages of [A_hi | A_lo | weight panel], each 1024-aligned
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t done;
@@ -66,7 +66,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     comp_gemm_kernel(const __grid_constant__ CUtensorMap tm_ahi, const __grid_constant__ CUtensorMap tm_alo,
                      const __grid_constant__ CUtensorMap tm_w, const int8_t* __restrict__ col_exp, float* y,
                      int64_t ld_y, const float* residual, int64_t ld_r, __half* gate_hi, __half* gate_lo,
-                     int64_t ld_g, int M, int N, int K, int box_rows, int* status, long long wait_ns) {
+                     int64_t ld_g, int M, int N, int K, int box_rows, int a_stride, int n_stages, int* status,
+                     long long wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -76,7 +77,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int ngroups = (nkb + GROUP_KB - 1) / GROUP_KB;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < n_stages; ++s) {
       inv::mbar_init(&sm.full[s], 1);
       inv::mbar_init(&sm.empty[s], 1);
     }
@@ -108,14 +109,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int nt = tile / tiles_m, mt = tile - nt * tiles_m;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!inv::mbar_wait(&sm.empty[stage], phase ^ 1u, wait_ns, abort_flag, status)) goto producer_done;
-          uint8_t* st = sm.stage[stage];
+          uint8_t* st = sm.ring + stage * (2 * a_stride + W_BYTES);
           inv::mbar_arrive_expect_tx(&sm.full[stage], 2 * a_bytes + W_BYTES);
           inv::tma_load_2d(st, &tm_ahi, &sm.full[stage], kb * BK, mt * BM);
-          inv::tma_load_2d(st + A_BYTES, &tm_alo, &sm.full[stage], kb * BK, mt * BM);
-          inv::tma_load_2d(st + 2 * A_BYTES, &tm_w, &sm.full[stage], kb * BK, nt * 2 * BN);
+          inv::tma_load_2d(st + a_stride, &tm_alo, &sm.full[stage], kb * BK, mt * BM);
+          inv::tma_load_2d(st + 2 * a_stride, &tm_w, &sm.full[stage], kb * BK, nt * 2 * BN);
           issued_mask |= 1u << stage;
           last_phase_mask = (last_phase_mask & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
+          if (++stage == (uint32_t)n_stages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -123,7 +124,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     producer_done:
       // Every load issued must have landed before the CTA may exit.
-      for (int s = 0; s < STAGES; ++s)
+      for (int s = 0; s < n_stages; ++s)
         if (issued_mask & (1u << s))
           inv::mbar_wait(&sm.full[s], (last_phase_mask >> s) & 1u, wait_ns, nullptr, status);
     }
@@ -142,17 +143,17 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int kb = kb0; kb < kb1; ++kb) {
             if (!inv::mbar_wait(&sm.full[stage], phase, wait_ns, abort_flag, status)) goto mma_done;
             inv::tc_fence_after();
-            const uint32_t base = inv::smem_u32(sm.stage[stage]);
+            const uint32_t base = inv::smem_u32(sm.ring + stage * (2 * a_stride + W_BYTES));
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
               const uint64_t ahi = inv::sw128_kmajor_desc(base + kk * 32);
-              const uint64_t alo = inv::sw128_kmajor_desc(base + A_BYTES + kk * 32);
-              const uint64_t bw = inv::sw128_kmajor_desc(base + 2 * A_BYTES + kk * 32);
+              const uint64_t alo = inv::sw128_kmajor_desc(base + a_stride + kk * 32);
+              const uint64_t bw = inv::sw128_kmajor_desc(base + 2 * a_stride + kk * 32);
               inv::umma_f16(d, ahi, bw, IDESC_N256, (kb > kb0 || kk > 0) ? 1u : 0u);
               inv::umma_f16(d + BN, alo, bw, IDESC_N128, 1u);
             }
             inv::umma_commit(&sm.empty[stage]);
-            if (++stage == STAGES) {
+            if (++stage == (uint32_t)n_stages) {
               stage = 0;
               phase ^= 1u;
             }
@@ -296,6 +297,13 @@ int launch_comp_gemm_ex(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, i
   if (M == 0) return INV_OK;
   // A rows per load: the whole 128-row tile, or only round_up(M, 8) when M < 128
   const int box_rows = M < BM ? (int)((M + 7) / 8 * 8) : BM;
+  // Stage = [A_hi | A_lo | weight panel]; with fewer A rows the same ring holds
+  // more stages (more weight bytes in flight).  The MMA still reads 128 A rows
+  // from each A base: rows past box_rows hold other data of the stage and
+  // only feed output rows that are never stored.
+  const int a_stride = (box_rows * BK * 2 + 1023) / 1024 * 1024;
+  const int stage_bytes = 2 * a_stride + W_BYTES;
+  const int n_stages = RING_BYTES / stage_bytes < MAX_STAGES ? RING_BYTES / stage_bytes : MAX_STAGES;
   CUtensorMap ta, tl, tw;
   int rc = make_tensor_map_2d(&ta, a_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)M,
                               (uint64_t)ld_a * 2, BK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -319,7 +327,7 @@ int launch_comp_gemm_ex(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, i
   comp_gemm_kernel<<<grid, THREADS, kSmemBytes, s>>>(ta, tl, tw, col_exp, y, ld_y, residual, ld_r,
                                                      reinterpret_cast<__half*>(gate_hi),
                                                      reinterpret_cast<__half*>(gate_lo), ld_g, (int)M, N, K,
-                                                     box_rows, status_ptr(), wait_limit_ns());
+                                                     box_rows, a_stride, n_stages, status_ptr(), wait_limit_ns());
   INV_CHECK_LAUNCH();
   return INV_OK;
 }
