@@ -461,14 +461,28 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o, const floa
   const int lane = threadIdx.x & 31;
   if (wid >= (int64_t)B * Hq) return;
   const int b = (int)(wid / Hq);
+  const float2* ml = part_ml + wid * S_max;
+  const float4* po = reinterpret_cast<const float4*>(part_o + wid * S_max * 128) + lane;
+  // The first 8 splits' (m, l) and o are requested together with len[b]: one
+  // memory round trip for KV lengths up to 2048.  Entries past the row's own
+  // split count are loaded (inside the partials buffer) but never used.
+  constexpr int PF = 8;
+  float2 v0[PF];
+  float4 o0[PF];
+#pragma unroll
+  for (int j = 0; j < PF; ++j) {
+    v0[j] = j < S_max ? ml[j] : make_float2(-INFINITY, 0.0f);
+    o0[j] = j < S_max ? po[j * 32] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   const int L = len[b];
   float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
   if (L >= 1 && L <= len_limit) {
     const int S = (L + SPLIT - 1) / SPLIT;
-    const float2* ml = part_ml + wid * S_max;
-    const float4* po = reinterpret_cast<const float4*>(part_o + wid * S_max * 128) + lane;
-    float M = -INFINITY;
-    for (int s0 = 0; s0 < S; s0 += 8) {  // exact max: order does not matter
+    float M = -INFINITY;  // exact max: order does not matter
+#pragma unroll
+    for (int j = 0; j < PF; ++j)
+      if (j < S) M = fmaxf(M, v0[j].x);
+    for (int s0 = PF; s0 < S; s0 += 8) {
       float2 v[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) v[j] = s0 + j < S ? ml[s0 + j] : make_float2(-INFINITY, 0.0f);
@@ -477,7 +491,18 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o, const floa
     }
     float l = 0.0f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0; s0 < S; s0 += 8) {  // splits folded in ascending order, 8 loads in flight
+    // splits folded in ascending order
+#pragma unroll
+    for (int j = 0; j < PF; ++j) {
+      if (j >= S) break;
+      const float f = expf(__fsub_rn(v0[j].x, M));
+      l = __fadd_rn(l, __fmul_rn(v0[j].y, f));
+      acc.x = __fadd_rn(acc.x, __fmul_rn(o0[j].x, f));
+      acc.y = __fadd_rn(acc.y, __fmul_rn(o0[j].y, f));
+      acc.z = __fadd_rn(acc.z, __fmul_rn(o0[j].z, f));
+      acc.w = __fadd_rn(acc.w, __fmul_rn(o0[j].w, f));
+    }
+    for (int s0 = PF; s0 < S; s0 += 8) {  // 8 loads in flight
       float2 v[8];
       float4 o[8];
 #pragma unroll
