@@ -45,6 +45,7 @@ sys.path.insert(0, ROOT)
 
 H, HQ, HKV, D, F = 4096, 32, 8, 128, 11008
 BATCH, KV_LEN = 128, 2048
+REFERENCE_SECONDS = 60.0  # timed oracle work of the reference arm, at most
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one attn_split launch per decoded row at KV length
 # 2048, from an ncu capture of the kernel at B = 32 (273.22 MB read + 6.92 MB
@@ -611,18 +612,28 @@ def run_reference(args, rank, world):
     p, cache, x = oracle_sample_inputs(rows)
     slot = np.arange(rows)
     pos = np.full(rows, KV_LEN - 1)
-    for _ in range(args.warmup):
+    # One step is one oracle decode_layer call on `rows` sequences (~0.1-0.3 s
+    # each).  So that the run stays within a few minutes whatever --steps is,
+    # warm-up is capped at 3 calls and the timed calls stop after ~60 s of
+    # oracle time; the line reports how many calls were timed.
+    warm = min(args.warmup, 3)
+    for _ in range(warm):
         ref.decode_layer(p, cache, x, slot, pos)
+    t_start = time.perf_counter()
     for _ in range(args.steps):
         t0 = time.perf_counter()
         ref.decode_layer(p, cache, x, slot, pos)
         times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_start > REFERENCE_SECONDS:
+            break
     ms = statistics.fmean(times) * 1e3
     v = rows / (ms * 1e-3)
-    sample = f"{rows} sequences per step (kv {KV_LEN}), float64 oracle decode_layer"
+    sample = (f"{len(times)} timed float64 oracle decode_layer calls of {rows} sequences (kv {KV_LEN}) "
+              f"for {args.steps} requested steps, {warm} warm-up calls")
     print(json.dumps({
         "impl": "reference", "metric": "batch-invariant decode-layer tokens/s", "value": round(v, 4),
-        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "unit": "tokens/s", "n_gpus": world, "steps": len(times), "steps_requested": args.steps,
+        "warmup": warm,
         "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"decode_layer H{H} Hq{HQ} Hkv{HKV} D{D} F{F} B{BATCH} kv{KV_LEN}",
