@@ -87,7 +87,7 @@ def test_decode_layer_full_shape_batch_invariance(inv):
     cfg = inv.LayerConfig(hidden=H, n_heads=HQ, n_kv_heads=HKV, ffn=F, max_pos=2048)
     w = inv.LayerWeights(cfg, wq, wk, wv, wo, wg, wu, wd, ga, gm)
     del wq, wk, wv, wo, wg, wu, wd
-    n_seq, ctx = 128, 2047
+    n_seq, ctx = 256, 2047
     cache = inv.KVCache(n_slots=n_seq, n_kv_heads=HKV, max_len=2048)
     for s in range(n_seq):
         sl = torch.full((ctx,), s, dtype=torch.int32, device="cuda")
@@ -97,7 +97,7 @@ def test_decode_layer_full_shape_batch_invariance(inv):
     x = torch.randn((n_seq, H), generator=g, device="cuda")
     pos = torch.full((n_seq,), ctx, dtype=torch.int32, device="cuda")
     ref_out = None
-    for B in (128, 32, 8, 1):
+    for B in (256, 128, 37, 8, 1):
         perm = torch.from_numpy(synth.permutation(n_seq, seed=B)).cuda()
         out = torch.empty_like(x)
         for a in range(0, n_seq, B):
