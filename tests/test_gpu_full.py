@@ -3,6 +3,8 @@
 * Decode layer at the 7B-like shape (hidden 4096, 32/8 heads of 128, MLP 11008,
   KV length 2048): oracle parity on sampled sequences, and per-sequence bit
   identity across batch sizes {1, 8, 32, 128} with shuffled composition.
+* prefill_layer versus decode_layer at that shape: identical bits per row and
+  an identical cache, chunk boundaries inside splits and row blocks.
 * Decode attention with 32/8 heads, B = 64, ragged lengths U(128, 8192), split
   256: oracle parity on sampled rows.
 * A layer stack with embedding, final RMSNorm, LM head (vocab 32000) and
@@ -107,6 +109,33 @@ def test_decode_layer_full_shape_batch_invariance(inv):
             ref_out = out
         else:
             assert torch.equal(out.view(torch.int32), ref_out.view(torch.int32)), B
+    assert status() == inv.INV_OK
+
+
+def test_prefill_layer_matches_decode_layer_full_shape(inv):
+    """At the 7B-like shape, prefill_layer (each split loaded once per 64-row
+    block) gives decode_layer's bits for every row and writes the same cache,
+    for chunks whose boundaries fall inside splits and row blocks."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(11)
+    mk = lambda *shape: torch.randn(shape, generator=g, device="cuda") * 0.02
+    cfg = inv.LayerConfig(hidden=H, n_heads=HQ, n_kv_heads=HKV, ffn=F, max_pos=1024)
+    w = inv.LayerWeights(cfg, mk(H, HQ * D), mk(H, HKV * D), mk(H, HKV * D), mk(HQ * D, H), mk(H, F), mk(H, F),
+                         mk(F, H), torch.rand(H, generator=g, device="cuda") + 0.5,
+                         torch.rand(H, generator=g, device="cuda") + 0.5)
+    xs = torch.randn((700, H), generator=g, device="cuda")
+    a = inv.KVCache(n_slots=2, n_kv_heads=HKV, max_len=1024)
+    b = inv.KVCache(n_slots=2, n_kv_heads=HKV, max_len=1024)
+    start = 0
+    for T in (300, 77, 323):
+        x = xs[start:start + T].contiguous()
+        pos = torch.arange(start, start + T, dtype=torch.int32, device="cuda")
+        y_dec = inv.decode_layer(cfg, w, a, x, torch.ones(T, dtype=torch.int32, device="cuda"), pos)
+        y_pre = inv.prefill_layer(cfg, w, b, x, 1, start)
+        assert torch.equal(y_dec.view(torch.int32), y_pre.view(torch.int32)), start
+        start += T
+    assert torch.equal(a.k, b.k) and torch.equal(a.v, b.v)
+    assert torch.equal(a.k_scale, b.k_scale) and torch.equal(a.v_scale, b.v_scale)
     assert status() == inv.INV_OK
 
 
