@@ -55,13 +55,19 @@ struct __align__(1024) DecodeSmem {
 };
 constexpr size_t kDecodeSmem = sizeof(DecodeSmem) + 1024;
 
+// Prefill: PF_GROUPS groups of 128 threads each run the per-row code on their
+// own rows of the block, so one SM keeps 4 x PF_GROUPS warps busy on the same
+// resident K and V.
+constexpr int PF_GROUPS = 4;
+constexpr int PF_THREADS = PF_GROUPS * THREADS;
+
 struct __align__(1024) PrefillSmem {
   uint8_t kcodes[CODE_BYTES];  // K and V of one split stay resident for every row
   uint8_t vcodes[CODE_BYTES];
-  float xo[4 * 4 * 128];       // warp exchange of O
+  float xo[PF_GROUPS][4 * 4 * 128];  // per group: warp exchange of O
   float ks[SPLIT];
   float vs[SPLIT];
-  RowScratch rs;
+  RowScratch rs[PF_GROUPS];
   uint64_t bar_kv;
   int abort;
 };
@@ -117,6 +123,9 @@ __device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
 
 // One query row of one split: the whole per-row computation shared by the
 // decode and prefill kernels, so a (row, split) gives the same bits in both.
+//   tid  : thread index within the row's 128-thread group.
+//   sync : barrier over exactly that group (__syncthreads in the decode kernel,
+//          a named barrier per group in the prefill kernel).
 //   qrow : fp32 q of the row's G query heads of this kv head ([G][128]).
 //   n    : valid keys of this row in the split (1..256); keys >= n are masked.
 //   kbase/vbase : shared addresses of the split's K / V codes (swizzled layout).
@@ -128,14 +137,14 @@ __device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
 //          overwrites only the codes of its own 64 keys); the decode kernel
 //          loads that warp's V codes into the warp's K slot there.
 //   out_o/out_ml : this row's partials for head 0 of the group, split s.
-template <bool kReuse, class IssueV, class WaitV>
-__device__ __forceinline__ void split_row(const float* __restrict__ qrow, int G, int n, uint32_t kbase,
+template <bool kReuse, class Sync, class IssueV, class WaitV>
+__device__ __forceinline__ void split_row(int tid, Sync sync, const float* __restrict__ qrow, int G, int n, uint32_t kbase,
                                           uint32_t vbase, const float* ks, const float* vs, RowScratch& rs,
                                           float* xo, float sigma, float* __restrict__ out_o,
                                           float2* __restrict__ out_ml, int64_t head_stride_o,
                                           int64_t head_stride_ml, bool ok, int* status, IssueV issue_v,
                                           WaitV wait_v) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
+  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
 
   // B fragments of S^T = K Q^T: column g is query head g/2 of the group, its
   // hi part for even g and lo part for odd g; rows k = d.
@@ -199,7 +208,7 @@ __device__ __forceinline__ void split_row(const float* __restrict__ qrow, int G,
   inv::fence_proxy_async_smem();  // this warp's K reads (generic proxy) before the TMA overwrite (async proxy)
   __syncwarp();
   issue_v();
-  __syncthreads();
+  sync();
 
   // ---------------------------------------------------------------- softmax --
   const float M = fmaxf(fmaxf(rs.red_m[0][c], rs.red_m[1][c]), fmaxf(rs.red_m[2][c], rs.red_m[3][c]));
@@ -226,7 +235,7 @@ __device__ __forceinline__ void split_row(const float* __restrict__ qrow, int G,
     rs.red_l[warp][c] = lsum;
     rs.red_w[warp][c] = wmax;
   }
-  __syncthreads();
+  sync();
   // per-(split, head) exponent E: max_j w_j 2^E in [2^14, 2^15)
   int E = 0;
   {
@@ -283,7 +292,7 @@ __device__ __forceinline__ void split_row(const float* __restrict__ qrow, int G,
     }
   }
   // o[dt]: (d = 16dt + g, col 2c = w_hi head c), (d, col 2c+1 = w_lo), (d+8, ...)
-  __syncthreads();  // every warp is done reading V codes (xo may alias them)
+  sync();  // every warp is done reading V codes (xo may alias them)
   const float unscale = inv::pow2f(-E);
 #pragma unroll
   for (int dt = 0; dt < 8; ++dt) {
@@ -292,7 +301,7 @@ __device__ __forceinline__ void split_row(const float* __restrict__ qrow, int G,
     xo[(warp * 4 + c) * 128 + 16 * dt + g] = v0;
     xo[(warp * 4 + c) * 128 + 16 * dt + g + 8] = v1;
   }
-  __syncthreads();
+  sync();
   for (int idx = tid; idx < 4 * 128; idx += THREADS) {
     const int head = idx >> 7, d = idx & 127;
     if (head >= G) continue;
@@ -310,7 +319,7 @@ __device__ __forceinline__ void split_row(const float* __restrict__ qrow, int G,
     l = __fadd_rn(l, rs.red_l[3][tid]);
     out_ml[tid * head_stride_ml] = make_float2(Mh, l);
   }
-  if (kReuse) __syncthreads();  // the scratch and xo are reused by the next row
+  if (kReuse) sync();  // the scratch and xo are reused by the next row
 }
 
 // Decode: one CTA per (row b, kv head h, split s).
@@ -367,7 +376,7 @@ __global__ void __launch_bounds__(THREADS, 3)
 
   bool v_issued = false;
   split_row<false>(
-      sm.qs, G, n, cbase, cbase, sm.ks, sm.vs, sm.rs, reinterpret_cast<float*>(sm.codes), sigma,
+      tid, []() { __syncthreads(); }, sm.qs, G, n, cbase, cbase, sm.ks, sm.vs, sm.rs, reinterpret_cast<float*>(sm.codes), sigma,
       part_o + (obase * S_max + s) * 128, part_ml + obase * S_max + s, (int64_t)S_max * 128, (int64_t)S_max, ok,
       status,
       [&]() {  // this warp is done with its K codes: bring its V codes into the same slot
@@ -393,10 +402,11 @@ __global__ void __launch_bounds__(THREADS, 3)
 // Prefill: rows r = 0..T-1 of one sequence (slot sl) at positions p0 + r.
 // One CTA per (kv head h, split s, block of ROWS_PER_CTA rows): the split's K
 // and V are loaded once and every row of the block that reaches split s runs
-// split_row -- the decode kernel's per-row code -- on them.
+// split_row -- the decode kernel's per-row code, with the same thread-to-data
+// mapping inside its 128-thread group -- on them, PF_GROUPS rows at a time.
 constexpr int ROWS_PER_CTA = 64;
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(PF_THREADS, 1)
     attn_prefill_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                               const float* __restrict__ q, const float* __restrict__ kscale,
                               const float* __restrict__ vscale, int sl, int p0, int T, int Hq, int Hkv, int max_len,
@@ -432,7 +442,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       inv::tma_load_2d(sm.vcodes + bx * 2 * BOX_BYTES + BOX_BYTES, &tm_v, &sm.bar_kv, 64, row0 + 64 * bx);
     }
   }
-  for (int j = tid; j < SPLIT; j += THREADS) {
+  for (int j = tid; j < SPLIT; j += PF_THREADS) {
     sm.ks[j] = j < n_max ? kscale[(int64_t)row0 + j] : 0.0f;
     sm.vs[j] = j < n_max ? vscale[(int64_t)row0 + j] : 0.0f;
   }
@@ -442,12 +452,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 
   const uint32_t kbase = inv::smem_u32(sm.kcodes), vbase = inv::smem_u32(sm.vcodes);
-  for (int r = r_first; r <= r_last; ++r) {
+  // group grp takes rows r_first + grp, r_first + grp + PF_GROUPS, ...; its
+  // barrier is named barrier 1 + grp over its own 128 threads
+  const int grp = tid / THREADS, gtid = tid % THREADS;
+  const auto group_sync = [grp]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(THREADS) : "memory"); };
+  for (int r = r_first + grp; r <= r_last; r += PF_GROUPS) {
     const int n = min(SPLIT, p0 + r + 1 - key0);
     const int64_t obase = (int64_t)r * Hq + (int64_t)h * G;
-    split_row<true>(q + obase * 128, G, n, kbase, vbase, sm.ks, sm.vs, sm.rs, sm.xo, sigma,
-              part_o + (obase * S_max + s) * 128, part_ml + obase * S_max + s, (int64_t)S_max * 128,
-              (int64_t)S_max, ok, status, []() {}, [](bool okv) { return okv; });
+    split_row<true>(gtid, group_sync, q + obase * 128, G, n, kbase, vbase, sm.ks, sm.vs, sm.rs[grp], sm.xo[grp],
+                    sigma, part_o + (obase * S_max + s) * 128, part_ml + obase * S_max + s, (int64_t)S_max * 128,
+                    (int64_t)S_max, ok, status, []() {}, [](bool okv) { return okv; });
   }
   if (tid == 0) inv::mbar_wait(&sm.bar_kv, 0, wait_ns, nullptr, status);
 }
@@ -619,7 +633,7 @@ int launch_attention_prefill(const float* q, int T, int Hq, const inv_kv_cache& 
   }
   dim3 grid(splits_for(pos0 + T), c.n_kv_heads, (T + ROWS_PER_CTA - 1) / ROWS_PER_CTA);
   trace_record(2 * trace_base, s);
-  attn_prefill_split_kernel<<<grid, THREADS, kPrefillSmem, s>>>(tk, tv, q, c.k_scale, c.v_scale, slot, pos0, T, Hq,
+  attn_prefill_split_kernel<<<grid, PF_THREADS, kPrefillSmem, s>>>(tk, tv, q, c.k_scale, c.v_scale, slot, pos0, T, Hq,
                                                                 c.n_kv_heads, c.max_len, S_max, sigma, part_o,
                                                                 part_ml, status_ptr(), wait_limit_ns());
   INV_CHECK_LAUNCH();
