@@ -195,10 +195,10 @@ def time_oracle(rows: int, min_seconds: float, max_calls: int = 1000):
 
 # ------------------------------------------------------------------- ours --
 
-def build_gpu_layer(inv, torch, device):
+def build_gpu_layer(inv, torch, device, max_pos=0):
     p = host_layer_params(0)
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
-    cfg = inv.LayerConfig(hidden=H, n_heads=HQ, n_kv_heads=HKV, ffn=F, max_pos=max(KV_LEN, 8192))
+    cfg = inv.LayerConfig(hidden=H, n_heads=HQ, n_kv_heads=HKV, ffn=F, max_pos=max(KV_LEN, 8192, max_pos))
     w = inv.LayerWeights(cfg, t(p.wq), t(p.wk), t(p.wv), t(p.wo), t(p.w_gate), t(p.w_up), t(p.w_down),
                          t(p.g_attn), t(p.g_mlp))
     return cfg, w
@@ -683,6 +683,39 @@ def run_gemm_only(args, local):
                       "steps": args.steps, "warmup": args.warmup}))
 
 
+def run_prefill_only(args, local):
+    """prefill_layer over one T-token sequence (one layer), one shot, timed with
+    CUDA events per call; one JSON line (for profiling the prefill kernels)."""
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    from invariant_numerics_b200 import build as _b
+    _b.build()
+    from invariant_numerics_b200 import invnum as inv
+    from invariant_numerics_b200 import synth
+    T = args.prefill
+    cfg, w = build_gpu_layer(inv, torch, device, max_pos=T)
+    x = torch.from_numpy(synth.normal((T, H), seed=77)).to(device)
+    y = torch.empty_like(x)
+    cache = inv.KVCache(n_slots=1, n_kv_heads=HKV, max_len=(T + 63) // 64 * 64, device=device)
+    ts = []
+    for i in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        inv.prefill_layer(cfg, w, cache, x, 0, 0, out=y)
+        b.record()
+        b.synchronize()
+        if i >= args.warmup:
+            ts.append(a.elapsed_time(b))
+    st = inv.inv_get_device_status()
+    if st != inv.INV_OK:
+        raise RuntimeError(f"device status {inv.status_string(st)}")
+    ms = statistics.median(ts)
+    print(json.dumps({"metric": "prefill_layer tokens/s", "value": round(T / (ms * 1e-3), 1), "unit": "tokens/s",
+                      "config": {"workload": f"prefill_layer H{H} Hq{HQ} Hkv{HKV} D{D} F{F} T{T} one-shot"},
+                      "ms": round(ms, 3), "steps": args.steps, "warmup": args.warmup}))
+
+
 def main():
     global BATCH, KV_LEN, H, HQ, HKV, F
     ap = argparse.ArgumentParser()
@@ -702,6 +735,8 @@ def main():
     ap.add_argument("--oracle-seconds", type=float, default=10.0)
     ap.add_argument("--gemm", type=int, nargs=3, metavar=("M", "N", "K"),
                     help="time one compensated GEMM shape only (one JSON line; for profiling)")
+    ap.add_argument("--prefill", type=int, metavar="T",
+                    help="time prefill_layer over one T-token sequence only (one JSON line; for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -714,6 +749,8 @@ def main():
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     if args.gemm:
         run_gemm_only(args, local)
+    elif args.prefill:
+        run_prefill_only(args, local)
     elif args.impl == "reference":
         run_reference(args, rank, world)
     else:

@@ -55,19 +55,21 @@ struct __align__(1024) DecodeSmem {
 };
 constexpr size_t kDecodeSmem = sizeof(DecodeSmem) + 1024;
 
-// Prefill: PF_GROUPS groups of 128 threads each run the per-row code on their
-// own rows of the block, so one SM keeps 4 x PF_GROUPS warps busy on the same
-// resident K and V.
+// Prefill: PF_GROUPS groups of 128 threads each run the per-row code on PF_R
+// rows at a time of the block (every unpacked K/V fragment feeds PF_R rows'
+// MMAs), so one SM keeps PF_GROUPS x PF_R rows in flight on the same resident
+// K and V.
 constexpr int PF_GROUPS = 4;
+constexpr int PF_R = 2;
 constexpr int PF_THREADS = PF_GROUPS * THREADS;
 
 struct __align__(1024) PrefillSmem {
   uint8_t kcodes[CODE_BYTES];  // K and V of one split stay resident for every row
   uint8_t vcodes[CODE_BYTES];
-  float xo[PF_GROUPS][4 * 4 * 128];  // per group: warp exchange of O
+  float xo[PF_GROUPS][PF_R][4 * 4 * 128];  // per group and row: warp exchange of O
   float ks[SPLIT];
   float vs[SPLIT];
-  RowScratch rs[PF_GROUPS];
+  RowScratch rs[PF_GROUPS][PF_R];
   uint64_t bar_kv;
   int abort;
 };
@@ -121,65 +123,88 @@ __device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
   return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
 }
 
-// One query row of one split: the whole per-row computation shared by the
-// decode and prefill kernels, so a (row, split) gives the same bits in both.
-//   tid  : thread index within the row's 128-thread group.
+// The query rows one call of split_rows works on: R rows of the same kv head
+// and split.  n[r] = 0 marks an absent row (nothing computed or written; its
+// q pointer must still be a readable row).
+template <int R>
+struct RowSet {
+  const float* q[R];      // fp32 q of the row's G query heads ([G][128])
+  int n[R];               // valid keys of the row in the split (0..256)
+  float* out_o[R];        // partial o of head 0 of the group, split s
+  float2* out_ml[R];      // partial (m, l) of head 0 of the group, split s
+};
+
+// R query rows of one split: the whole per-row computation shared by the
+// decode (R = 1) and prefill (R = 2) kernels.  Each unpacked K or V fragment
+// feeds the MMAs of all R rows, and every row's accumulators receive exactly
+// the MMAs, in exactly the order, that they receive with R = 1 (an m-tile
+// beyond a row's n is skipped for that row), so a (row, split) gives the same
+// bits in both kernels.
+//   tid  : thread index within the rows' 128-thread group.
 //   sync : barrier over exactly that group (__syncthreads in the decode kernel,
 //          a named barrier per group in the prefill kernel).
-//   qrow : fp32 q of the row's G query heads of this kv head ([G][128]).
-//   n    : valid keys of this row in the split (1..256); keys >= n are masked.
 //   kbase/vbase : shared addresses of the split's K / V codes (swizzled layout).
 //   ks/vs : shared scales (zero beyond the keys that were loaded).
-//   xo   : shared [4 warps][4 heads][128] exchange buffer (may alias the codes
-//          in the decode kernel: it is written only after the last V read).
+//   rs   : R scratch records, one per row.
+//   xo   : R shared [4 warps][4 heads][128] exchange buffers (in the decode
+//          kernel the one buffer aliases the codes: it is written only after
+//          the last V read).
 //   issue_v / wait_v : hooks around the first V access.  issue_v runs in every
 //          thread once its warp has finished reading K (a warp reads and later
 //          overwrites only the codes of its own 64 keys); the decode kernel
 //          loads that warp's V codes into the warp's K slot there.
-//   out_o/out_ml : this row's partials for head 0 of the group, split s.
-template <bool kReuse, class Sync, class IssueV, class WaitV>
-__device__ __forceinline__ void split_row(int tid, Sync sync, const float* __restrict__ qrow, int G, int n, uint32_t kbase,
-                                          uint32_t vbase, const float* ks, const float* vs, RowScratch& rs,
-                                          float* xo, float sigma, float* __restrict__ out_o,
-                                          float2* __restrict__ out_ml, int64_t head_stride_o,
-                                          int64_t head_stride_ml, bool ok, int* status, IssueV issue_v,
-                                          WaitV wait_v) {
+template <int R, bool kReuse, class Sync, class IssueV, class WaitV>
+__device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& rows, int G, uint32_t kbase,
+                                           uint32_t vbase, const float* ks, const float* vs, RowScratch* rs,
+                                           float* xo, float sigma, int64_t head_stride_o, int64_t head_stride_ml,
+                                           bool ok, int* status, IssueV issue_v, WaitV wait_v) {
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
+  int n_max = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) n_max = max(n_max, rows.n[r]);
 
   // B fragments of S^T = K Q^T: column g is query head g/2 of the group, its
   // hi part for even g and lo part for odd g; rows k = d.
-  uint32_t qf[8][2];
+  uint32_t qf[R][8][2];
   {
     const int head = g >> 1;
     const bool lo = (g & 1) != 0;
-    const bool valid = head < G;
-    const float* qh = qrow + head * 128;
     bool bad = false;
 #pragma unroll
-    for (int ks_ = 0; ks_ < 8; ++ks_) {
+    for (int r = 0; r < R; ++r) {
+      const bool valid = head < G && rows.n[r] > 0;
+      const float* qh = rows.q[r] + head * 128;
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int d = 16 * ks_ + 2 * c + 8 * r;
-        const float x0 = valid ? qh[d] : 0.0f, x1 = valid ? qh[d + 1] : 0.0f;
-        __half h0, l0, h1, l1;
-        inv::split_hi_lo(x0, h0, l0);
-        inv::split_hi_lo(x1, h1, l1);
-        bad |= inv::f16_overflow(x0) | inv::f16_overflow(x1);
-        qf[ks_][r] = lo ? pack_half2(l0, l1) : pack_half2(h0, h1);
+      for (int ks_ = 0; ks_ < 8; ++ks_) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int d = 16 * ks_ + 2 * c + 8 * i;
+          const float x0 = valid ? qh[d] : 0.0f, x1 = valid ? qh[d + 1] : 0.0f;
+          __half h0, l0, h1, l1;
+          inv::split_hi_lo(x0, h0, l0);
+          inv::split_hi_lo(x1, h1, l1);
+          bad |= inv::f16_overflow(x0) | inv::f16_overflow(x1);
+          qf[r][ks_][i] = lo ? pack_half2(l0, l1) : pack_half2(h0, h1);
+        }
       }
     }
     if (bad) record_status(status, INV_ERR_RANGE);
   }
 
   // ---------------------------------------------------------------- scores --
-  float tsc[4][2];
-  float mx = -INFINITY;
+  float tsc[R][4][2];
+  float mx[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) mx[r] = -INFINITY;
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt) {
     const int kb = warp * 64 + mt * 16;
-    tsc[mt][0] = tsc[mt][1] = -INFINITY;
-    if (ok && kb < n) {
-      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int r = 0; r < R; ++r) tsc[r][mt][0] = tsc[r][mt][1] = -INFINITY;
+    if (ok && kb < n_max) {
+      float acc[R][4];
+#pragma unroll
+      for (int r = 0; r < R; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.0f;
       const int lkey = kb + ((lane >> 3) & 1) * 8 + (lane & 7);
 #pragma unroll
       for (int ks_ = 0; ks_ < 8; ++ks_) {
@@ -187,98 +212,124 @@ __device__ __forceinline__ void split_row(int tid, Sync sync, const float* __res
         ldsm_x4(code_addr(kbase, lkey, 16 * ks_ + (lane >> 4) * 8), a);
 #pragma unroll
         for (int i = 0; i < 4; ++i) unpack_dual(a[i], ah[i], al[i]);
-        mma16816(acc, ah, qf[ks_][0], qf[ks_][1]);
-        mma16816(acc, al, qf[ks_][0], qf[ks_][1]);
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+          if (kb < rows.n[r]) mma16816(acc[r], ah, qf[r][ks_][0], qf[r][ks_][1]);
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+          if (kb < rows.n[r]) mma16816(acc[r], al, qf[r][ks_][0], qf[r][ks_][1]);
       }
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int key = kb + g + 8 * r;
-        // acc[2r] = q_hi . code / 256, acc[2r+1] = q_lo . code / 256 (head c)
-        const float dot = __fmul_rn(__fadd_rn(acc[2 * r], __fmul_rn(acc[2 * r + 1], 0x1p-11f)), 256.0f);
-        const float t = __fmul_rn(__fmul_rn(dot, ks[key]), sigma);
-        tsc[mt][r] = key < n ? t : -INFINITY;
-        mx = fmaxf(mx, tsc[mt][r]);
+      for (int r = 0; r < R; ++r) {
+        if (kb >= rows.n[r]) continue;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int key = kb + g + 8 * i;
+          // acc[2i] = q_hi . code / 256, acc[2i+1] = q_lo . code / 256 (head c)
+          const float dot = __fmul_rn(__fadd_rn(acc[r][2 * i], __fmul_rn(acc[r][2 * i + 1], 0x1p-11f)), 256.0f);
+          const float t = __fmul_rn(__fmul_rn(dot, ks[key]), sigma);
+          tsc[r][mt][i] = key < rows.n[r] ? t : -INFINITY;
+          mx[r] = fmaxf(mx[r], tsc[r][mt][i]);
+        }
       }
     }
   }
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-  if (g == 0) rs.red_m[warp][c] = mx;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 4));
+    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 8));
+    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 16));
+    if (g == 0) rs[r].red_m[warp][c] = mx[r];
+  }
   inv::fence_proxy_async_smem();  // this warp's K reads (generic proxy) before the TMA overwrite (async proxy)
   __syncwarp();
   issue_v();
   sync();
 
   // ---------------------------------------------------------------- softmax --
-  const float M = fmaxf(fmaxf(rs.red_m[0][c], rs.red_m[1][c]), fmaxf(rs.red_m[2][c], rs.red_m[3][c]));
-  float w[4][2];
-  float lsum = 0.0f, wmax = 0.0f;
+  float w[R][4][2];
+  int E[R];
+  {
+    float lsum[R], wmax[R];
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt) {
+    for (int r = 0; r < R; ++r) {
+      const float M = fmaxf(fmaxf(rs[r].red_m[0][c], rs[r].red_m[1][c]), fmaxf(rs[r].red_m[2][c], rs[r].red_m[3][c]));
+      lsum[r] = 0.0f;
+      wmax[r] = 0.0f;
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int key = warp * 64 + mt * 16 + g + 8 * r;
-      const float p = tsc[mt][r] == -INFINITY ? 0.0f : expf(__fsub_rn(tsc[mt][r], M));
-      lsum = __fadd_rn(lsum, p);
-      w[mt][r] = (key < n && p != 0.0f) ? __fmul_rn(p, vs[key]) : 0.0f;
-      wmax = fmaxf(wmax, w[mt][r]);
+      for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int key = warp * 64 + mt * 16 + g + 8 * i;
+          const float p = tsc[r][mt][i] == -INFINITY ? 0.0f : expf(__fsub_rn(tsc[r][mt][i], M));
+          lsum[r] = __fadd_rn(lsum[r], p);
+          w[r][mt][i] = (key < rows.n[r] && p != 0.0f) ? __fmul_rn(p, vs[key]) : 0.0f;
+          wmax[r] = fmaxf(wmax[r], w[r][mt][i]);
+        }
+      }
+      lsum[r] = __fadd_rn(lsum[r], __shfl_xor_sync(0xffffffffu, lsum[r], 4));
+      lsum[r] = __fadd_rn(lsum[r], __shfl_xor_sync(0xffffffffu, lsum[r], 8));
+      lsum[r] = __fadd_rn(lsum[r], __shfl_xor_sync(0xffffffffu, lsum[r], 16));
+      wmax[r] = fmaxf(wmax[r], __shfl_xor_sync(0xffffffffu, wmax[r], 4));
+      wmax[r] = fmaxf(wmax[r], __shfl_xor_sync(0xffffffffu, wmax[r], 8));
+      wmax[r] = fmaxf(wmax[r], __shfl_xor_sync(0xffffffffu, wmax[r], 16));
+      if (g == 0) {
+        rs[r].red_l[warp][c] = lsum[r];
+        rs[r].red_w[warp][c] = wmax[r];
+      }
     }
   }
-  lsum = __fadd_rn(lsum, __shfl_xor_sync(0xffffffffu, lsum, 4));
-  lsum = __fadd_rn(lsum, __shfl_xor_sync(0xffffffffu, lsum, 8));
-  lsum = __fadd_rn(lsum, __shfl_xor_sync(0xffffffffu, lsum, 16));
-  wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, 4));
-  wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, 8));
-  wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, 16));
-  if (g == 0) {
-    rs.red_l[warp][c] = lsum;
-    rs.red_w[warp][c] = wmax;
-  }
   sync();
-  // per-(split, head) exponent E: max_j w_j 2^E in [2^14, 2^15)
-  int E = 0;
-  {
-    const float wm = fmaxf(fmaxf(rs.red_w[0][c], rs.red_w[1][c]), fmaxf(rs.red_w[2][c], rs.red_w[3][c]));
+  // per-(split, head) exponent E: max_j w_j 2^E in [2^14, 2^15); packed
+  // (hi, lo) of w 2^E for keys g and g+8 of every m-tile
+  uint32_t pw_hi[R][4], pw_lo[R][4];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    E[r] = 0;
+    const float wm = fmaxf(fmaxf(rs[r].red_w[0][c], rs[r].red_w[1][c]), fmaxf(rs[r].red_w[2][c], rs[r].red_w[3][c]));
     if (wm > 0.0f) {
       int ex;
       frexpf(wm, &ex);
-      E = 15 - ex;
-      E = E < -120 ? -120 : (E > 120 ? 120 : E);
+      E[r] = 15 - ex;
+      E[r] = E[r] < -120 ? -120 : (E[r] > 120 ? 120 : E[r]);
     }
-  }
-  const float scaleE = inv::pow2f(E);
-  // packed (hi, lo) of w 2^E for keys g and g+8 of every m-tile
-  uint32_t pw_hi[4], pw_lo[4];
+    const float scaleE = inv::pow2f(E[r]);
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt) {
-    __half h0, l0, h1, l1;
-    inv::split_hi_lo(__fmul_rn(w[mt][0], scaleE), h0, l0);
-    inv::split_hi_lo(__fmul_rn(w[mt][1], scaleE), h1, l1);
-    pw_hi[mt] = pack_half2(h0, h1);
-    pw_lo[mt] = pack_half2(l0, l1);
+    for (int mt = 0; mt < 4; ++mt) {
+      __half h0, l0, h1, l1;
+      inv::split_hi_lo(__fmul_rn(w[r][mt][0], scaleE), h0, l0);
+      inv::split_hi_lo(__fmul_rn(w[r][mt][1], scaleE), h1, l1);
+      pw_hi[r][mt] = pack_half2(h0, h1);
+      pw_lo[r][mt] = pack_half2(l0, l1);
+    }
   }
 
   ok = wait_v(ok);
 
   // --------------------------------------------------------------- values --
-  float o[8][4];
+  float o[R][8][4];
 #pragma unroll
-  for (int dt = 0; dt < 8; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.0f;
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int dt = 0; dt < 8; ++dt) o[r][dt][0] = o[r][dt][1] = o[r][dt][2] = o[r][dt][3] = 0.0f;
   const int src1 = 4 * (2 * c) + (g >> 1), src2 = 4 * (2 * c + 1) + (g >> 1);
   const bool want_lo = (g & 1) != 0;
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt) {
     const int kb = warp * 64 + mt * 16;
     // B fragment of O^T = V^T W: rows k = keys, column g = head g/2 (hi/lo)
-    const uint32_t x1h = __shfl_sync(0xffffffffu, pw_hi[mt], src1);
-    const uint32_t x1l = __shfl_sync(0xffffffffu, pw_lo[mt], src1);
-    const uint32_t x2h = __shfl_sync(0xffffffffu, pw_hi[mt], src2);
-    const uint32_t x2l = __shfl_sync(0xffffffffu, pw_lo[mt], src2);
-    const uint32_t x1 = want_lo ? x1l : x1h, x2 = want_lo ? x2l : x2h;
-    const uint32_t b0 = __byte_perm(x1, x2, 0x5410);  // keys 2c, 2c+1
-    const uint32_t b1 = __byte_perm(x1, x2, 0x7632);  // keys 2c+8, 2c+9
-    if (ok && kb < n) {
+    uint32_t b0[R], b1[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const uint32_t x1h = __shfl_sync(0xffffffffu, pw_hi[r][mt], src1);
+      const uint32_t x1l = __shfl_sync(0xffffffffu, pw_lo[r][mt], src1);
+      const uint32_t x2h = __shfl_sync(0xffffffffu, pw_hi[r][mt], src2);
+      const uint32_t x2l = __shfl_sync(0xffffffffu, pw_lo[r][mt], src2);
+      const uint32_t x1 = want_lo ? x1l : x1h, x2 = want_lo ? x2l : x2h;
+      b0[r] = __byte_perm(x1, x2, 0x5410);  // keys 2c, 2c+1
+      b1[r] = __byte_perm(x1, x2, 0x7632);  // keys 2c+8, 2c+9
+    }
+    if (ok && kb < n_max) {
       const int lkey = kb + (lane >> 4) * 8 + (lane & 7);
 #pragma unroll
       for (int dt = 0; dt < 8; ++dt) {
@@ -286,40 +337,56 @@ __device__ __forceinline__ void split_row(int tid, Sync sync, const float* __res
         ldsm_x4_t(code_addr(vbase, lkey, 16 * dt + ((lane >> 3) & 1) * 8), a);
 #pragma unroll
         for (int i = 0; i < 4; ++i) unpack_dual(a[i], ah[i], al[i]);
-        mma16816(o[dt], ah, b0, b1);
-        mma16816(o[dt], al, b0, b1);
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+          if (kb < rows.n[r]) mma16816(o[r][dt], ah, b0[r], b1[r]);
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+          if (kb < rows.n[r]) mma16816(o[r][dt], al, b0[r], b1[r]);
       }
     }
   }
-  // o[dt]: (d = 16dt + g, col 2c = w_hi head c), (d, col 2c+1 = w_lo), (d+8, ...)
+  // o[r][dt]: (d = 16dt + g, col 2c = w_hi head c), (d, col 2c+1 = w_lo), (d+8, ...)
   sync();  // every warp is done reading V codes (xo may alias them)
-  const float unscale = inv::pow2f(-E);
 #pragma unroll
-  for (int dt = 0; dt < 8; ++dt) {
-    const float v0 = __fmul_rn(__fmul_rn(__fadd_rn(o[dt][0], __fmul_rn(o[dt][1], 0x1p-11f)), 256.0f), unscale);
-    const float v1 = __fmul_rn(__fmul_rn(__fadd_rn(o[dt][2], __fmul_rn(o[dt][3], 0x1p-11f)), 256.0f), unscale);
-    xo[(warp * 4 + c) * 128 + 16 * dt + g] = v0;
-    xo[(warp * 4 + c) * 128 + 16 * dt + g + 8] = v1;
+  for (int r = 0; r < R; ++r) {
+    const float unscale = inv::pow2f(-E[r]);
+    float* xr = xo + r * (4 * 4 * 128);
+#pragma unroll
+    for (int dt = 0; dt < 8; ++dt) {
+      const float v0 =
+          __fmul_rn(__fmul_rn(__fadd_rn(o[r][dt][0], __fmul_rn(o[r][dt][1], 0x1p-11f)), 256.0f), unscale);
+      const float v1 =
+          __fmul_rn(__fmul_rn(__fadd_rn(o[r][dt][2], __fmul_rn(o[r][dt][3], 0x1p-11f)), 256.0f), unscale);
+      xr[(warp * 4 + c) * 128 + 16 * dt + g] = v0;
+      xr[(warp * 4 + c) * 128 + 16 * dt + g + 8] = v1;
+    }
   }
   sync();
-  for (int idx = tid; idx < 4 * 128; idx += THREADS) {
-    const int head = idx >> 7, d = idx & 127;
-    if (head >= G) continue;
-    float v = xo[(0 * 4 + head) * 128 + d];
-    v = __fadd_rn(v, xo[(1 * 4 + head) * 128 + d]);
-    v = __fadd_rn(v, xo[(2 * 4 + head) * 128 + d]);
-    v = __fadd_rn(v, xo[(3 * 4 + head) * 128 + d]);
-    out_o[head * head_stride_o + d] = v;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (rows.n[r] <= 0) continue;
+    const float* xr = xo + r * (4 * 4 * 128);
+    for (int idx = tid; idx < 4 * 128; idx += THREADS) {
+      const int head = idx >> 7, d = idx & 127;
+      if (head >= G) continue;
+      float v = xr[(0 * 4 + head) * 128 + d];
+      v = __fadd_rn(v, xr[(1 * 4 + head) * 128 + d]);
+      v = __fadd_rn(v, xr[(2 * 4 + head) * 128 + d]);
+      v = __fadd_rn(v, xr[(3 * 4 + head) * 128 + d]);
+      rows.out_o[r][head * head_stride_o + d] = v;
+    }
+    if (tid < G) {
+      const RowScratch& sr = rs[r];
+      const float Mh = fmaxf(fmaxf(sr.red_m[0][tid], sr.red_m[1][tid]), fmaxf(sr.red_m[2][tid], sr.red_m[3][tid]));
+      float l = sr.red_l[0][tid];
+      l = __fadd_rn(l, sr.red_l[1][tid]);
+      l = __fadd_rn(l, sr.red_l[2][tid]);
+      l = __fadd_rn(l, sr.red_l[3][tid]);
+      rows.out_ml[r][tid * head_stride_ml] = make_float2(Mh, l);
+    }
   }
-  if (tid < G) {
-    const float Mh = fmaxf(fmaxf(rs.red_m[0][tid], rs.red_m[1][tid]), fmaxf(rs.red_m[2][tid], rs.red_m[3][tid]));
-    float l = rs.red_l[0][tid];
-    l = __fadd_rn(l, rs.red_l[1][tid]);
-    l = __fadd_rn(l, rs.red_l[2][tid]);
-    l = __fadd_rn(l, rs.red_l[3][tid]);
-    out_ml[tid * head_stride_ml] = make_float2(Mh, l);
-  }
-  if (kReuse) sync();  // the scratch and xo are reused by the next row
+  if (kReuse) sync();  // the scratch and xo are reused by the next rows
 }
 
 // Decode: one CTA per (row b, kv head h, split s).
@@ -375,10 +442,10 @@ __global__ void __launch_bounds__(THREADS, 3)
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 
   bool v_issued = false;
-  split_row<false>(
-      tid, []() { __syncthreads(); }, sm.qs, G, n, cbase, cbase, sm.ks, sm.vs, sm.rs, reinterpret_cast<float*>(sm.codes), sigma,
-      part_o + (obase * S_max + s) * 128, part_ml + obase * S_max + s, (int64_t)S_max * 128, (int64_t)S_max, ok,
-      status,
+  const RowSet<1> rows = {{sm.qs}, {n}, {part_o + (obase * S_max + s) * 128}, {part_ml + obase * S_max + s}};
+  split_rows<1, false>(
+      tid, []() { __syncthreads(); }, rows, G, cbase, cbase, sm.ks, sm.vs, &sm.rs,
+      reinterpret_cast<float*>(sm.codes), sigma, (int64_t)S_max * 128, (int64_t)S_max, ok, status,
       [&]() {  // this warp is done with its K codes: bring its V codes into the same slot
         const int warp = tid >> 5;
         if (lane == 0 && ok && warp < nbox) {
@@ -402,8 +469,9 @@ __global__ void __launch_bounds__(THREADS, 3)
 // Prefill: rows r = 0..T-1 of one sequence (slot sl) at positions p0 + r.
 // One CTA per (kv head h, split s, block of ROWS_PER_CTA rows): the split's K
 // and V are loaded once and every row of the block that reaches split s runs
-// split_row -- the decode kernel's per-row code, with the same thread-to-data
-// mapping inside its 128-thread group -- on them, PF_GROUPS rows at a time.
+// split_rows -- the decode kernel's per-row code, with the same thread-to-data
+// mapping inside its 128-thread group -- on them, PF_GROUPS x PF_R rows at a
+// time.
 constexpr int ROWS_PER_CTA = 64;
 
 __global__ void __launch_bounds__(PF_THREADS, 1)
@@ -452,16 +520,24 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 
   const uint32_t kbase = inv::smem_u32(sm.kcodes), vbase = inv::smem_u32(sm.vcodes);
-  // group grp takes rows r_first + grp, r_first + grp + PF_GROUPS, ...; its
-  // barrier is named barrier 1 + grp over its own 128 threads
+  // group grp takes the rows r0 .. r0 + PF_R - 1 for r0 = r_first + grp PF_R,
+  // then + PF_GROUPS PF_R, ...; its barrier is named barrier 1 + grp over its
+  // own 128 threads.  A row past r_last is absent (n = 0).
   const int grp = tid / THREADS, gtid = tid % THREADS;
   const auto group_sync = [grp]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(THREADS) : "memory"); };
-  for (int r = r_first + grp; r <= r_last; r += PF_GROUPS) {
-    const int n = min(SPLIT, p0 + r + 1 - key0);
-    const int64_t obase = (int64_t)r * Hq + (int64_t)h * G;
-    split_row<true>(gtid, group_sync, q + obase * 128, G, n, kbase, vbase, sm.ks, sm.vs, sm.rs[grp], sm.xo[grp],
-                    sigma, part_o + (obase * S_max + s) * 128, part_ml + obase * S_max + s, (int64_t)S_max * 128,
-                    (int64_t)S_max, ok, status, []() {}, [](bool okv) { return okv; });
+  for (int r0 = r_first + grp * PF_R; r0 <= r_last; r0 += PF_GROUPS * PF_R) {
+    RowSet<PF_R> rows;
+#pragma unroll
+    for (int i = 0; i < PF_R; ++i) {
+      const int r = r0 + i <= r_last ? r0 + i : r0;
+      const int64_t obase = (int64_t)r * Hq + (int64_t)h * G;
+      rows.q[i] = q + obase * 128;
+      rows.n[i] = r0 + i <= r_last ? min(SPLIT, p0 + r + 1 - key0) : 0;
+      rows.out_o[i] = part_o + (obase * S_max + s) * 128;
+      rows.out_ml[i] = part_ml + obase * S_max + s;
+    }
+    split_rows<PF_R, true>(gtid, group_sync, rows, G, kbase, vbase, sm.ks, sm.vs, sm.rs[grp], sm.xo[grp][0], sigma,
+                           (int64_t)S_max * 128, (int64_t)S_max, ok, status, []() {}, [](bool okv) { return okv; });
   }
   if (tid == 0) inv::mbar_wait(&sm.bar_kv, 0, wait_ns, nullptr, status);
 }
