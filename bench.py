@@ -48,10 +48,10 @@ BATCH, KV_LEN = 128, 2048
 REFERENCE_SECONDS = 60.0  # timed oracle work of the reference arm, at most
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one attn_split launch per decoded row at KV length
-# 2048, from an ncu capture of the kernel at B = 32 (273.22 MB read + 6.92 MB
+# 2048, from an ncu capture of the kernel at B = 32 (273.22 MB read + 6.08 MB
 # written), scaled by rows.  Set to None whenever the kernel changes and the
 # capture has not been repeated.
-ATTN_SPLIT_DRAM_BYTES_PER_ROW_KV2048 = (273.218560e6 + 6.921984e6) / 32
+ATTN_SPLIT_DRAM_BYTES_PER_ROW_KV2048 = (273.222656e6 + 6.080512e6) / 32
 
 
 def load_peaks():
