@@ -62,15 +62,58 @@ struct __align__(1024) GemmSmem {
 };
 constexpr size_t kSmemBytes = sizeof(GemmSmem) + 1024;
 
+// Consumer side of a producer/consumer GEMM pair: ready_row[kb] counts the
+// epilogue warps of the producing grid that have stored (and released) the
+// 64 A columns of K block kb of this row tile; EPI_WARPS means complete.
+// Scans forward from kb, a window of 64 counters per memory round trip, as
+// far as the blocks are complete; on success *upto is the end of that run
+// (> kb) and the acquire and async-proxy fences that make the data visible to
+// this thread's TMA loads have been executed once for the whole run.  Gives
+// up like mbar_wait (time limit or *abort).
+__device__ bool wait_published(const int* ready_row, int kb, int nkb, int* upto, long long limit_ns,
+                               volatile int* abort, int* status) {
+  constexpr int WIN = 64;
+  const unsigned long long t0 = inv::global_ns();
+  for (uint32_t i = 0;; ++i) {
+    int end = kb;  // first block not seen complete
+    for (;;) {
+      uint64_t done = 0;
+#pragma unroll
+      for (int j = 0; j < WIN; ++j) {
+        const int v = end + j < nkb ? inv::ld_relaxed_gpu(ready_row + end + j) : 0;
+        done |= (uint64_t)(v == EPI_WARPS) << j;
+      }
+      const int run = ~done == 0 ? WIN : __ffsll((long long)~done) - 1;
+      end += run;
+      if (run < WIN || end >= nkb) break;
+    }
+    if (end > kb) {
+      inv::fence_acquire_gpu();
+      inv::fence_proxy_async_global();
+      *upto = end;
+      return true;
+    }
+    if (abort != nullptr && *abort) return false;
+    if ((i & 15u) == 15u && (long long)(inv::global_ns() - t0) > limit_ns) {
+      inv::record_status(status, INV_ERR_TIMEOUT);
+      if (abort != nullptr) *abort = 1;
+      return false;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
     comp_gemm_kernel(const __grid_constant__ CUtensorMap tm_ahi, const __grid_constant__ CUtensorMap tm_alo,
                      const __grid_constant__ CUtensorMap tm_w, const int8_t* __restrict__ col_exp, float* y,
                      int64_t ld_y, const float* residual, int64_t ld_r, __half* gate_hi, __half* gate_lo,
-                     int64_t ld_g, int M, int N, int K, int box_rows, int a_stride, int n_stages, int* status,
-                     long long wait_ns) {
+                     int64_t ld_g, int M, int N, int K, int box_rows, int a_stride, int n_stages, int* ready_out,
+                     const int* ready_in, int* status, long long wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // A grid that publishes its tiles lets its consumer grid start as soon as
+  // every one of its own CTAs is resident (the consumer waits per K block).
+  if (ready_out != nullptr) inv::grid_launch_dependents();
   const int tiles_m = (M + BM - 1) / BM;
   const int n_tiles = tiles_m * (N / BN);
   const int nkb = K / BK;
@@ -105,10 +148,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t a_bytes = (uint32_t)box_rows * (BK * 2);  // one of A_hi / A_lo
       uint32_t stage = 0, phase = 0;
       uint32_t issued_mask = 0, last_phase_mask = 0;
+      int ready_mt = -1, ready_upto = 0;  // K blocks [0, ready_upto) of row tile ready_mt seen published
       for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
         const int nt = tile / tiles_m, mt = tile - nt * tiles_m;
+        if (mt != ready_mt) {
+          ready_mt = mt;
+          ready_upto = 0;
+        }
         for (int kb = 0; kb < nkb; ++kb) {
           if (!inv::mbar_wait(&sm.empty[stage], phase ^ 1u, wait_ns, abort_flag, status)) goto producer_done;
+          if (ready_in != nullptr && kb >= ready_upto &&
+              !wait_published(ready_in + (int64_t)mt * nkb, kb, nkb, &ready_upto, wait_ns, abort_flag, status))
+            goto producer_done;
           uint8_t* st = sm.ring + stage * (2 * a_stride + W_BYTES);
           inv::mbar_arrive_expect_tx(&sm.full[stage], 2 * a_bytes + W_BYTES);
           inv::tma_load_2d(st, &tm_ahi, &sm.full[stage], kb * BK, mt * BM);
@@ -265,6 +316,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
+      if (ready_out != nullptr) {
+        // publish: this warp's stores of the tile, then one release add per
+        // warp; the tile is complete when all EPI_WARPS warps have added
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) inv::red_release_gpu_add(ready_out + (int64_t)mt * (N / BN) + nt, 1);
+      }
     }
   epi_done:;
   }
@@ -275,6 +333,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     inv::tc_fence_after();
     inv::tmem_dealloc(tmem, TMEM_COLS);
   }
+  // a consumer grid completes only after its producer grid has
+  if (ready_in != nullptr) inv::grid_wait_prerequisites();
 }
 
 bool g_attr_set[64] = {};
@@ -287,13 +347,13 @@ int launch_comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int 
                      const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
                      const float* residual, int64_t ld_r, cudaStream_t s) {
   return launch_comp_gemm_ex(a_hi, a_lo, M, K, ld_a, w_packed, col_exp, N, y, ld_y, residual, ld_r, nullptr, nullptr,
-                             0, s);
+                             0, nullptr, nullptr, s);
 }
 
 int launch_comp_gemm_ex(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
                         const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
                         const float* residual, int64_t ld_r, uint16_t* gate_hi, uint16_t* gate_lo, int64_t ld_g,
-                        cudaStream_t s) {
+                        int* ready_out, const int* ready_in, cudaStream_t s) {
   if (M == 0) return INV_OK;
   // A rows per load: the whole 128-row tile, or only round_up(M, 8) when M < 128
   const int box_rows = M < BM ? (int)((M + 7) / 8 * 8) : BM;
@@ -324,10 +384,24 @@ int launch_comp_gemm_ex(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, i
   }
   const int64_t tiles = ((M + BM - 1) / BM) * (N / BN);
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-  comp_gemm_kernel<<<grid, THREADS, kSmemBytes, s>>>(ta, tl, tw, col_exp, y, ld_y, residual, ld_r,
-                                                     reinterpret_cast<__half*>(gate_hi),
-                                                     reinterpret_cast<__half*>(gate_lo), ld_g, (int)M, N, K,
-                                                     box_rows, a_stride, n_stages, status_ptr(), wait_limit_ns());
+  // A consumer (ready_in) is launched as a programmatic dependent of the
+  // producer launched just before it on the stream, so it may start while the
+  // producer's last tiles are still running; it waits per K block instead.
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(grid);
+  lc.blockDim = dim3(THREADS);
+  lc.dynamicSmemBytes = kSmemBytes;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = ready_in != nullptr ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&lc, comp_gemm_kernel, ta, tl, tw, col_exp, y, ld_y, residual, ld_r,
+                                           reinterpret_cast<__half*>(gate_hi), reinterpret_cast<__half*>(gate_lo),
+                                           ld_g, (int)M, N, K, box_rows, a_stride, n_stages, ready_out, ready_in,
+                                           status_ptr(), wait_limit_ns());
+  if (e != cudaSuccess) return INV_ERR_CUDA;
   INV_CHECK_LAUNCH();
   return INV_OK;
 }

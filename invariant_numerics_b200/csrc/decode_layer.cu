@@ -25,6 +25,7 @@ struct LayerWs {
   float* x1;
   uint16_t *h2_hi, *h2_lo;
   uint16_t *a_hi, *a_lo;
+  int* ready;          // gate/up tiles published to the down GEMM
   size_t bytes;
 };
 
@@ -54,6 +55,7 @@ LayerWs carve(const inv_layer_config& c, int B, int mlb, uint8_t* base) {
   w.h2_lo = reinterpret_cast<uint16_t*>(take(B * H * 2));
   w.a_hi = reinterpret_cast<uint16_t*>(take(B * F * 2));
   w.a_lo = reinterpret_cast<uint16_t*>(take(B * F * 2));
+  w.ready = reinterpret_cast<int*>(take(inv::gemm_ready_bytes(B, (int)(2 * F))));
   w.bytes = off;
   return w;
 }
@@ -128,10 +130,14 @@ int run_layer(const inv_layer_config* cfg, const inv_layer_weights* w, const inv
   // 7. h2 = rmsnorm(x1) -> hi/lo
   INV_TRACED(6, inv::launch_rmsnorm(ws.x1, w->g_mlp, B, H, cfg->eps, nullptr, ws.h2_hi, ws.h2_lo, s));
   // 8-9. [gate | up] = h2 W_gu with the SwiGLU a = silu(gate) * up fused in the epilogue -> hi/lo
+  // 10. out = x1 + a W_down.  The down GEMM starts while the gate/up GEMM's
+  // last tiles (a partial wave) run, loading each 64-column K block of a as
+  // soon as the gate/up tile that stores it has published it.
+  if (cudaMemsetAsync(ws.ready, 0, inv::gemm_ready_bytes(B, 2 * F), s) != cudaSuccess) return INV_ERR_CUDA;
   INV_TRACED(7, inv::launch_comp_gemm_ex(ws.h2_hi, ws.h2_lo, B, H, H, w->w_gu, w->e_gu, 2 * F, nullptr, 0, nullptr, 0,
-                                         ws.a_hi, ws.a_lo, F, s));
-  // 10. out = x1 + a W_down
-  INV_TRACED(8, inv::launch_comp_gemm(ws.a_hi, ws.a_lo, B, F, F, w->w_down, w->e_down, H, x_out, H, ws.x1, H, s));
+                                         ws.a_hi, ws.a_lo, F, ws.ready, nullptr, s));
+  INV_TRACED(8, inv::launch_comp_gemm_ex(ws.a_hi, ws.a_lo, B, F, F, w->w_down, w->e_down, H, x_out, H, ws.x1, H,
+                                         nullptr, nullptr, 0, nullptr, ws.ready, s));
 #undef INV_TRACED
   return INV_OK;
 }

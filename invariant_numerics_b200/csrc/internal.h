@@ -25,10 +25,20 @@ int launch_comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int 
 // columns interleaved in groups of 16 ([gate 16 | up 16] per 32 columns);
 // writes the hi/lo split of silu(gate) * up to gate_hi/gate_lo [M][ld_g]
 // (N/2 outputs per row) instead of y.
+// Producer/consumer pair (both nullable): a producer given ready_out
+// ([tiles_m][N/128] ints, zero before the launch) adds 1 per epilogue warp to
+// ready_out[mt][nt] once that warp has stored its part of tile (mt, nt); a
+// consumer given ready_in (the producer's array; the producer's N/128 must
+// equal the consumer's K/64) is launched as a programmatic dependent of the
+// producer launched just before it on the same stream and loads K block kb of
+// row tile mt only once ready_in[mt][kb] is complete.  Neither changes the
+// arithmetic.
 int launch_comp_gemm_ex(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
                         const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
                         const float* residual, int64_t ld_r, uint16_t* gate_hi, uint16_t* gate_lo, int64_t ld_g,
-                        cudaStream_t s);
+                        int* ready_out, const int* ready_in, cudaStream_t s);
+// Bytes of the ready array of a producer GEMM with M rows and N columns.
+inline size_t gemm_ready_bytes(int64_t M, int N) { return (size_t)((M + 127) / 128) * (size_t)(N / 128) * 4; }
 
 // Workspace layout of the attention: partial (m, l) and partial o per
 // (row, head, split).
