@@ -59,9 +59,10 @@ def _rounding_relevant_fp32():
 def test_rn16_matches_numpy_cast_on_every_rounding_boundary():
     x = _rounding_relevant_fp32()
     with warnings.catch_warnings():
-        warnings.simplefilter("ignore")
+        warnings.simplefilter("ignore")              # signalling NaNs among the random bit patterns
         want = x.astype(np.float16).view(np.uint16)
-    got = enc.rn16_bits(x.astype(np.float64))
+        xd = x.astype(np.float64)
+    got = enc.rn16_bits(xd)
     bad = np.nonzero(got != want)[0]
     assert bad.size == 0, [(float(x[i]), hex(int(got[i])), hex(int(want[i]))) for i in bad[:5]]
 
@@ -70,9 +71,10 @@ def test_rn16_matches_numpy_cast_on_random_fp32():
     r = np.random.Generator(np.random.PCG64(1234)).integers(0, 2**32, size=1 << 21, dtype=np.uint64)
     x = r.astype(np.uint32).view(np.float32)
     with warnings.catch_warnings():
-        warnings.simplefilter("ignore")
+        warnings.simplefilter("ignore")              # signalling NaNs among the random bit patterns
         want = x.astype(np.float16).view(np.uint16)
-    got = enc.rn16_bits(x.astype(np.float64))
+        xd = x.astype(np.float64)
+    got = enc.rn16_bits(xd)
     ok = (got == want) | np.isnan(x)
     assert ok.all()
 
