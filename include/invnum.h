@@ -279,6 +279,13 @@ INV_API int rmsnorm_bi(const float* x, const float* gamma, int64_t rows, int hid
  *   slot, pos   : int32 [B]; 0 <= pos[b] < min(cache->max_len, cfg->max_pos).
  *   rope_cos, rope_sin : fp32 [max_pos][64], cos/sin(p * base^(-2i/128)).
  *   workspace   : >= decode_layer_workspace_size(cfg, B, max_len_bound) bytes.
+ *                 Calls that overlap on the GPU need separate workspaces.
+ * Stream work: one memset of the workspace's gate/up tile counters and the
+ * layer's kernels, all on `stream`.  The W_down GEMM is launched as a
+ * programmatic dependent of the gate/up GEMM and starts during its last
+ * partial wave, loading each K block of a once the gate/up tile that stores it
+ * has published it (no change to any product or sum).  All of this may be
+ * captured into a CUDA graph.
  * Errors: as the component calls; INV_ERR_WORKSPACE.
  * ------------------------------------------------------------------------ */
 typedef struct {
