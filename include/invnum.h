@@ -100,6 +100,20 @@ INV_API int inv_set_wait_limit_ns(long long ns);
 INV_API int inv_selftest_wait_timeout(long long wait_ns, inv_stream stream);
 
 /*
+ * Self-test of the bounded wait of a GEMM consumer (the W_down GEMM of
+ * decode_layer waits on per-tile counters of the gate/up GEMM): launches a
+ * small consumer GEMM whose one input block is never published, with a limit
+ * of `wait_ns` nanoseconds.  It must give up, record INV_ERR_TIMEOUT and exit.
+ * `workspace`: >= INV_SELFTEST_GEMM_WS_BYTES of caller device memory, 16-byte
+ * aligned (cleared and used for the operands).  For failure-detection tests.
+ * Errors: INV_ERR_INVALID_ARG (wait_ns <= 0, null or misaligned workspace),
+ * INV_ERR_WORKSPACE.
+ */
+#define INV_SELFTEST_GEMM_WS_BYTES 40192u
+INV_API int inv_selftest_gemm_wait_timeout(void* workspace, size_t ws_bytes, long long wait_ns,
+                                           inv_stream stream);
+
+/*
  * Kernel tracing for decode_layer (profiling aid; off by default).  With
  * events != NULL and n_events >= 2 * INV_DECODE_LAYER_KERNELS, every later
  * decode_layer call records events[2i] before and events[2i+1] after its i-th
@@ -210,7 +224,10 @@ INV_API int kv_quant_int16(const float* x, int T, int64_t ld_x, const int32_t* s
  *   split    : must equal INV_KV_SPLIT.
  *   out      : fp32 [B][n_heads][128]; out_hi/out_lo: binary16 split of out
  *              (both NULL or both non-NULL).
- *   workspace: >= attn_decode_workspace_size(B, n_heads, max_len_bound) bytes.
+ *   workspace: >= attn_decode_workspace_size(B, n_heads, L) bytes, where L is
+ *              the bound the call resolves to: min(max_len_bound,
+ *              cache->max_len), or cache->max_len when max_len_bound <= 0.
+ *              The size function itself needs L > 0 (it returns 0 otherwise).
  * Errors: INV_ERR_INVALID_ARG; INV_ERR_UNSUPPORTED_SHAPE unless head_dim == 128
  * and n_heads / n_kv_heads is 1, 2 or 4; INV_ERR_WORKSPACE.
  * Device: INV_ERR_INVALID_ARG for a len/slot out of range (row skipped),
@@ -230,9 +247,10 @@ INV_API int attn_decode_fixedsplit(const float* q, int B, int n_heads, const inv
  * synchronise the device).  No counterpart on the pages: it is an interface
  * variant only.  The split partials live in a file-scope device array of
  * INV_NOALLOC_SCRATCH_BYTES on every GPU that loads the library, held until
- * exit.  Calls needing more than that (attn_decode_workspace_size(B, n_heads,
- * max_len_bound) > INV_NOALLOC_SCRATCH_BYTES) return INV_ERR_WORKSPACE and
- * launch nothing.  The first call on a device looks the array's address up
+ * exit.  Calls needing more than that return INV_ERR_WORKSPACE and launch
+ * nothing: the test is attn_decode_workspace_size(B, n_heads, L) >
+ * INV_NOALLOC_SCRATCH_BYTES with the resolved bound L = min(max_len_bound,
+ * cache->max_len), or L = cache->max_len when max_len_bound <= 0.  The first call on a device looks the array's address up
  * (with that device current); make it before any stream capture.  All calls on
  * a device share the array, so calls that overlap on the GPU race; calls
  * ordered on one stream do not.  Allocates nothing; arguments and other errors
@@ -278,8 +296,11 @@ INV_API int rmsnorm_bi(const float* x, const float* gamma, int64_t rows, int hid
  *   x_in, x_out : fp32 [B][hidden] (may not alias).
  *   slot, pos   : int32 [B]; 0 <= pos[b] < min(cache->max_len, cfg->max_pos).
  *   rope_cos, rope_sin : fp32 [max_pos][64], cos/sin(p * base^(-2i/128)).
- *   workspace   : >= decode_layer_workspace_size(cfg, B, max_len_bound) bytes.
- *                 Calls that overlap on the GPU need separate workspaces.
+ *   workspace   : >= decode_layer_workspace_size(cfg, B, L) bytes, L the
+ *                 resolved bound: min(max_len_bound, cache->max_len), or
+ *                 cache->max_len when max_len_bound <= 0 (the size function
+ *                 returns 0 for L <= 0).  Calls that overlap on the GPU need
+ *                 separate workspaces.
  * Stream work: one memset of the workspace's gate/up tile counters and the
  * layer's kernels, all on `stream`.  The W_down GEMM is launched as a
  * programmatic dependent of the gate/up GEMM and starts during its last
@@ -327,7 +348,8 @@ INV_API int decode_layer(const inv_layer_config* cfg, const inv_layer_weights* w
  * chunked prefill and decode must not change a row's reduction).
  *   x_in, x_out : fp32 [T][hidden].  0 <= slot < n_slots; 0 <= pos0;
  *   pos0 + T <= min(max_len_bound (or cache->max_len), cfg->max_pos).
- *   workspace : >= prefill_layer_workspace_size(cfg, T, max_len_bound) bytes.
+ *   workspace : >= prefill_layer_workspace_size(cfg, T, L) bytes, L resolved
+ *               as for decode_layer.
  * Errors: as decode_layer.
  * ------------------------------------------------------------------------ */
 INV_API size_t prefill_layer_workspace_size(const inv_layer_config* cfg, int T, int max_len_bound);

@@ -35,20 +35,25 @@
 namespace {
 
 constexpr int BM = INV_GEMM_BM;            // 128
-constexpr int BN = INV_GEMM_BN;            // 128
 constexpr int BK = INV_GEMM_BK;            // 64
 constexpr int MAX_STAGES = 8;
-constexpr int RING_BYTES = 3 * (2 * BM * INV_GEMM_BK * 2 + 2 * INV_GEMM_BN * INV_GEMM_BK * 2);  // 192 KB
+constexpr int RING_BYTES = 3 * (2 * BM * INV_GEMM_BK * 2 + 2 * 128 * INV_GEMM_BK * 2);  // 192 KB
 constexpr int GROUP_KB = INV_GEMM_KGROUP / BK;  // 4
-constexpr int W_BYTES = 2 * BN * BK * 2;   // 32 KB: 128 hi rows then 128 lo rows
-constexpr int ACC_COLS = 2 * BN;           // hh | cross
-constexpr int TMEM_COLS = 2 * ACC_COLS;    // two group buffers
 constexpr int EPI_WARPS = 8;
-constexpr int EPI_COLS = BN / 2;           // output columns per epilogue thread
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
-constexpr uint32_t IDESC_N256 = inv::idesc_f16_f32(128, 256);
-constexpr uint32_t IDESC_N128 = inv::idesc_f16_f32(128, 128);
-static_assert(TMEM_COLS <= 512, "tensor memory holds 512 columns");
+
+// Everything that depends on the panel width BN (output columns per tile).
+template <int BN>
+struct Tile {
+  static_assert(BN == 32 || BN == 64 || BN == 128, "panel widths 32, 64, 128");
+  static constexpr int W_BYTES = 2 * BN * BK * 2;   // BN hi rows then BN lo rows, 64 K each
+  static constexpr int ACC_COLS = 2 * BN;           // hh | cross
+  static constexpr int TMEM_COLS = 2 * ACC_COLS;    // two group buffers
+  static constexpr int EPI_COLS = BN / 2;           // output columns per epilogue thread
+  static constexpr uint32_t IDESC_HILO = inv::idesc_f16_f32(128, 2 * BN);
+  static constexpr uint32_t IDESC_HI = inv::idesc_f16_f32(128, BN);
+  static_assert(TMEM_COLS <= 512, "tensor memory holds 512 columns");
+};
 
 struct __align__(1024) GemmSmem {
   uint8_t ring[RING_BYTES];  // n_stages stages of [A_hi | A_lo | weight panel], each 1024-aligned
@@ -102,12 +107,15 @@ __device__ bool wait_published(const int* ready_row, int kb, int nkb, int* upto,
   }
 }
 
+template <int BN>
 __global__ void __launch_bounds__(THREADS, 1)
     comp_gemm_kernel(const __grid_constant__ CUtensorMap tm_ahi, const __grid_constant__ CUtensorMap tm_alo,
                      const __grid_constant__ CUtensorMap tm_w, const int8_t* __restrict__ col_exp, float* y,
                      int64_t ld_y, const float* residual, int64_t ld_r, __half* gate_hi, __half* gate_lo,
                      int64_t ld_g, int M, int N, int K, int box_rows, int a_stride, int n_stages, int* ready_out,
                      const int* ready_in, int* status, long long wait_ns) {
+  using T = Tile<BN>;
+  constexpr int W_BYTES = T::W_BYTES, ACC_COLS = T::ACC_COLS, TMEM_COLS = T::TMEM_COLS, EPI_COLS = T::EPI_COLS;
   extern __shared__ uint8_t smem_raw[];
   GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -200,8 +208,8 @@ __global__ void __launch_bounds__(THREADS, 1)
               const uint64_t ahi = inv::sw128_kmajor_desc(base + kk * 32);
               const uint64_t alo = inv::sw128_kmajor_desc(base + a_stride + kk * 32);
               const uint64_t bw = inv::sw128_kmajor_desc(base + 2 * a_stride + kk * 32);
-              inv::umma_f16(d, ahi, bw, IDESC_N256, (kb > kb0 || kk > 0) ? 1u : 0u);
-              inv::umma_f16(d + BN, alo, bw, IDESC_N128, 1u);
+              inv::umma_f16(d, ahi, bw, T::IDESC_HILO, (kb > kb0 || kk > 0) ? 1u : 0u);
+              inv::umma_f16(d + BN, alo, bw, T::IDESC_HI, 1u);
             }
             inv::umma_commit(&sm.empty[stage]);
             if (++stage == (uint32_t)n_stages) {
@@ -256,9 +264,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int col0 = nt * BN + half * EPI_COLS;
         if (row < M && gate_hi != nullptr) {
           // Fused SwiGLU: each 32 packed columns are 16 gate columns then the
-          // 16 matching up columns of outputs f0 .. f0+15, f0 = column / 2.
+          // 16 matching up columns of outputs f0 .. f0+15, f0 = column / 2
+          // (a panel of BN >= 64 columns; the host never asks for less).
 #pragma unroll
-          for (int c = 0; c < EPI_COLS; c += 32) {
+          for (int c = 0; c < (EPI_COLS % 32 == 0 ? EPI_COLS : 0); c += 32) {
             const int f0 = (col0 + c) / 2;
             float v[32];
 #pragma unroll
@@ -337,24 +346,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (ready_in != nullptr) inv::grid_wait_prerequisites();
 }
 
-bool g_attr_set[64] = {};
-
-}  // namespace
-
-namespace inv {
-
-int launch_comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
-                     const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
-                     const float* residual, int64_t ld_r, cudaStream_t s) {
-  return launch_comp_gemm_ex(a_hi, a_lo, M, K, ld_a, w_packed, col_exp, N, y, ld_y, residual, ld_r, nullptr, nullptr,
-                             0, nullptr, nullptr, s);
-}
-
-int launch_comp_gemm_ex(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
-                        const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
-                        const float* residual, int64_t ld_r, uint16_t* gate_hi, uint16_t* gate_lo, int64_t ld_g,
-                        int* ready_out, const int* ready_in, cudaStream_t s) {
-  if (M == 0) return INV_OK;
+// One launch of the BN-wide kernel (arguments validated by the caller).
+template <int BN>
+int launch_tiles(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a, const uint16_t* w_packed,
+                 const int8_t* col_exp, int N, float* y, int64_t ld_y, const float* residual, int64_t ld_r,
+                 uint16_t* gate_hi, uint16_t* gate_lo, int64_t ld_g, int* ready_out, const int* ready_in,
+                 cudaStream_t s, long long wait_ns) {
+  static bool attr_set[64] = {};
   // A rows per load: the whole 128-row tile, or only round_up(M, 8) when M < 128
   const int box_rows = M < BM ? (int)((M + 7) / 8 * 8) : BM;
   // Stage = [A_hi | A_lo | weight panel]; with fewer A rows the same ring holds
@@ -362,28 +360,28 @@ int launch_comp_gemm_ex(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, i
   // from each A base: rows past box_rows hold other data of the stage and
   // only feed output rows that are never stored.
   const int a_stride = (box_rows * BK * 2 + 1023) / 1024 * 1024;
-  const int stage_bytes = 2 * a_stride + W_BYTES;
+  const int stage_bytes = 2 * a_stride + Tile<BN>::W_BYTES;
   const int n_stages = RING_BYTES / stage_bytes < MAX_STAGES ? RING_BYTES / stage_bytes : MAX_STAGES;
   CUtensorMap ta, tl, tw;
-  int rc = make_tensor_map_2d(&ta, a_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)M,
-                              (uint64_t)ld_a * 2, BK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+  int rc = inv::make_tensor_map_2d(&ta, a_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)M,
+                                   (uint64_t)ld_a * 2, BK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != INV_OK) return rc;
-  rc = make_tensor_map_2d(&tl, a_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)M, (uint64_t)ld_a * 2,
-                          BK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+  rc = inv::make_tensor_map_2d(&tl, a_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)M,
+                               (uint64_t)ld_a * 2, BK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != INV_OK) return rc;
-  rc = make_tensor_map_2d(&tw, w_packed, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)N * 2,
-                          (uint64_t)K * 2, BK, 2 * BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  rc = inv::make_tensor_map_2d(&tw, w_packed, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (uint64_t)K, (uint64_t)N * 2,
+                               (uint64_t)K * 2, BK, 2 * BN, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != INV_OK) return rc;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !g_attr_set[dev]) {
-    if (cudaFuncSetAttribute(comp_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(comp_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
         cudaSuccess)
       return INV_ERR_CUDA;
-    g_attr_set[dev] = true;
+    attr_set[dev] = true;
   }
   const int64_t tiles = ((M + BM - 1) / BM) * (N / BN);
-  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  const int grid = (int)(tiles < inv::sm_count() ? tiles : inv::sm_count());
   // A consumer (ready_in) is launched as a programmatic dependent of the
   // producer launched just before it on the stream, so it may start while the
   // producer's last tiles are still running; it waits per K block instead.
@@ -397,13 +395,49 @@ int launch_comp_gemm_ex(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, i
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = ready_in != nullptr ? 1 : 0;
-  const cudaError_t e = cudaLaunchKernelEx(&lc, comp_gemm_kernel, ta, tl, tw, col_exp, y, ld_y, residual, ld_r,
+  const cudaError_t e = cudaLaunchKernelEx(&lc, comp_gemm_kernel<BN>, ta, tl, tw, col_exp, y, ld_y, residual, ld_r,
                                            reinterpret_cast<__half*>(gate_hi), reinterpret_cast<__half*>(gate_lo),
                                            ld_g, (int)M, N, K, box_rows, a_stride, n_stages, ready_out, ready_in,
-                                           status_ptr(), wait_limit_ns());
+                                           inv::status_ptr(), wait_ns < 0 ? inv::wait_limit_ns() : wait_ns);
   if (e != cudaSuccess) return INV_ERR_CUDA;
   INV_CHECK_LAUNCH();
   return INV_OK;
+}
+
+}  // namespace
+
+namespace inv {
+
+int gemm_panel_width(int N) {
+  (void)N;
+  return INV_GEMM_BN;
+}
+
+int launch_comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
+                     const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
+                     const float* residual, int64_t ld_r, cudaStream_t s) {
+  return launch_comp_gemm_ex(a_hi, a_lo, M, K, ld_a, w_packed, col_exp, N, y, ld_y, residual, ld_r, nullptr, nullptr,
+                             0, nullptr, nullptr, s);
+}
+
+int launch_comp_gemm_ex(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
+                        const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
+                        const float* residual, int64_t ld_r, uint16_t* gate_hi, uint16_t* gate_lo, int64_t ld_g,
+                        int* ready_out, const int* ready_in, cudaStream_t s, long long wait_ns) {
+  if (M == 0) return INV_OK;
+  switch (gemm_panel_width(N)) {
+    case 128:
+      return launch_tiles<128>(a_hi, a_lo, M, K, ld_a, w_packed, col_exp, N, y, ld_y, residual, ld_r, gate_hi, gate_lo,
+                               ld_g, ready_out, ready_in, s, wait_ns);
+    case 64:
+      return launch_tiles<64>(a_hi, a_lo, M, K, ld_a, w_packed, col_exp, N, y, ld_y, residual, ld_r, gate_hi, gate_lo,
+                              ld_g, ready_out, ready_in, s, wait_ns);
+    case 32:
+      return launch_tiles<32>(a_hi, a_lo, M, K, ld_a, w_packed, col_exp, N, y, ld_y, residual, ld_r, gate_hi, gate_lo,
+                              ld_g, ready_out, ready_in, s, wait_ns);
+    default:
+      return INV_ERR_UNSUPPORTED_SHAPE;
+  }
 }
 
 }  // namespace inv
@@ -412,7 +446,7 @@ extern "C" int comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, 
                          const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
                          const float* residual, int64_t ld_r, inv_stream stream) {
   if (M < 0 || K <= 0 || N <= 0) return INV_ERR_INVALID_ARG;
-  if (K % BK != 0 || N % BN != 0) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (K % BK != 0 || N % inv::gemm_panel_width(N) != 0) return INV_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return INV_OK;
   if (M > 0x7fffffffLL) return INV_ERR_UNSUPPORTED_SHAPE;
   if (!a_hi || !a_lo || !w_packed || !col_exp || !y) return INV_ERR_INVALID_ARG;
@@ -423,4 +457,27 @@ extern "C" int comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, 
   if ((reinterpret_cast<uintptr_t>(col_exp) & 3u) != 0) return INV_ERR_INVALID_ARG;
   return inv::launch_comp_gemm(a_hi, a_lo, M, K, ld_a, w_packed, col_exp, N, y, ld_y, residual, ld_r,
                                static_cast<cudaStream_t>(stream));
+}
+
+// Self-test of the consumer side of a GEMM pair: a small consumer GEMM (M = 8,
+// K = 64, N = 128) whose one K block is never published (its counter is
+// zeroed and no producer runs) must give up after wait_ns, record
+// INV_ERR_TIMEOUT and exit.  The operands live in the caller's workspace;
+// their values do not matter (nothing is loaded).
+extern "C" int inv_selftest_gemm_wait_timeout(void* workspace, size_t ws_bytes, long long wait_ns,
+                                              inv_stream stream) {
+  if (wait_ns <= 0 || workspace == nullptr || !inv::aligned16(workspace)) return INV_ERR_INVALID_ARG;
+  if (ws_bytes < INV_SELFTEST_GEMM_WS_BYTES) return INV_ERR_WORKSPACE;
+  constexpr int M = 8, K = 64, N = 128;
+  uint8_t* p = static_cast<uint8_t*>(workspace);
+  uint16_t* a_hi = reinterpret_cast<uint16_t*>(p);                 // [8][64] binary16
+  uint16_t* a_lo = reinterpret_cast<uint16_t*>(p + 1024);
+  uint16_t* w = reinterpret_cast<uint16_t*>(p + 2048);             // [1][2][128][64] binary16
+  int8_t* e = reinterpret_cast<int8_t*>(p + 2048 + 32768);         // [128]
+  float* y = reinterpret_cast<float*>(p + 2048 + 32768 + 256);     // [8][128]
+  int* ready = reinterpret_cast<int*>(p + 2048 + 32768 + 256 + 4096);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, INV_SELFTEST_GEMM_WS_BYTES, s) != cudaSuccess) return INV_ERR_CUDA;
+  return inv::launch_comp_gemm_ex(a_hi, a_lo, M, K, K, w, e, N, y, N, nullptr, 0, nullptr, nullptr, 0, nullptr, ready,
+                                  s, wait_ns);
 }

@@ -147,9 +147,12 @@ int run_layer(const inv_layer_config* cfg, const inv_layer_weights* w, const inv
 extern "C" {
 
 size_t decode_layer_workspace_size(const inv_layer_config* cfg, int B, int max_len_bound) {
-  if (!cfg || B <= 0 || cfg->hidden <= 0 || cfg->ffn <= 0 || cfg->n_heads <= 0 || cfg->n_kv_heads <= 0) return 0;
-  const int mlb = max_len_bound > 0 ? max_len_bound : 1;
-  return carve(*cfg, B, mlb, nullptr).bytes;
+  // The bound must be the one the call resolves to (a positive bound, or the
+  // cache's max_len when the call passes <= 0); <= 0 here has no size.
+  if (!cfg || B <= 0 || max_len_bound <= 0 || cfg->hidden <= 0 || cfg->ffn <= 0 || cfg->n_heads <= 0 ||
+      cfg->n_kv_heads <= 0)
+    return 0;
+  return carve(*cfg, B, max_len_bound, nullptr).bytes;
 }
 
 int decode_layer(const inv_layer_config* cfg, const inv_layer_weights* w, const inv_kv_cache* cache,

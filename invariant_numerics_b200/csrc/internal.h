@@ -17,6 +17,10 @@ int launch_rope_quant(const float* qkv, int T, int Hq, const inv_kv_cache& c, co
                       int32_t* len_out, cudaStream_t s);
 
 
+// Panel width (output columns per GEMM tile and per packed panel) of a weight
+// with N output columns: a function of N alone, so every M uses the same tile.
+int gemm_panel_width(int N);
+
 int launch_comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
                      const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
                      const float* residual, int64_t ld_r, cudaStream_t s);
@@ -32,11 +36,11 @@ int launch_comp_gemm(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int 
 // equal the consumer's K/64) is launched as a programmatic dependent of the
 // producer launched just before it on the same stream and loads K block kb of
 // row tile mt only once ready_in[mt][kb] is complete.  Neither changes the
-// arithmetic.
+// arithmetic.  wait_ns < 0: the library-wide wait bound.
 int launch_comp_gemm_ex(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
                         const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
                         const float* residual, int64_t ld_r, uint16_t* gate_hi, uint16_t* gate_lo, int64_t ld_g,
-                        int* ready_out, const int* ready_in, cudaStream_t s);
+                        int* ready_out, const int* ready_in, cudaStream_t s, long long wait_ns = -1);
 // Bytes of the ready array of a producer GEMM with M rows and N columns.
 inline size_t gemm_ready_bytes(int64_t M, int N) { return (size_t)((M + 127) / 128) * (size_t)(N / 128) * 4; }
 

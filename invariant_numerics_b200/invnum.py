@@ -57,6 +57,7 @@ _SIGS = {
     "inv_get_device_status": (_i, [C.POINTER(_i), _p]),
     "inv_set_wait_limit_ns": (_i, [C.c_longlong]),
     "inv_selftest_wait_timeout": (_i, [C.c_longlong, _p]),
+    "inv_selftest_gemm_wait_timeout": (_i, [_p, _sz, C.c_longlong, _p]),
     "inv_trace_events": (_i, [C.POINTER(C.c_void_p), _i]),
     "heal_split": (_i, [_p, _i64, _i64, _i64, _p, _p, _i64, _p]),
     "heal_packed_weight_bytes": (_sz, [_i, _i]),
@@ -99,6 +100,12 @@ def _ptr(t):
     return None if t is None else C.c_void_p(t.data_ptr())
 
 
+def _resolved_bound(cache, max_len_bound: int) -> int:
+    """The KV length bound a call resolves to (the C entry points' rule): the
+    caller's bound clipped to the cache, or the cache's max_len for <= 0."""
+    return cache.max_len if max_len_bound <= 0 else min(max_len_bound, cache.max_len)
+
+
 def _need(t, dtype, name, contiguous=True):
     if t is None:
         raise ValueError(f"{name} is required")
@@ -129,6 +136,15 @@ def inv_set_wait_limit_ns(ns: int) -> None:
 
 def inv_selftest_wait_timeout(wait_ns: int, stream=None) -> None:
     _check("inv_selftest_wait_timeout", lib.inv_selftest_wait_timeout(int(wait_ns), _stream(stream)))
+
+
+SELFTEST_GEMM_WS_BYTES = 40192
+
+
+def inv_selftest_gemm_wait_timeout(wait_ns: int, workspace=None, stream=None) -> None:
+    ws = torch.empty(SELFTEST_GEMM_WS_BYTES, dtype=torch.uint8, device="cuda") if workspace is None else workspace
+    _check("inv_selftest_gemm_wait_timeout",
+           lib.inv_selftest_gemm_wait_timeout(_ptr(ws), ws.numel(), int(wait_ns), _stream(stream)))
 
 
 DECODE_LAYER_KERNELS = 9
@@ -236,7 +252,7 @@ def attn_decode_fixedsplit(q, cache: KVCache, slot, lens, softmax_scale, max_len
     out = torch.empty_like(q) if out is None else _need(out, torch.float32, "out")
     hi = torch.empty(q.shape, dtype=torch.float16, device=q.device) if want_split else None
     lo = torch.empty(q.shape, dtype=torch.float16, device=q.device) if want_split else None
-    nbytes = lib.attn_decode_workspace_size(B, Hq, min(mlb, cache.max_len))
+    nbytes = lib.attn_decode_workspace_size(B, Hq, _resolved_bound(cache, mlb))
     if workspace is None:
         workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=q.device)
     cs = cache.struct()
@@ -382,7 +398,7 @@ def decode_layer(cfg: LayerConfig, w: LayerWeights, cache: KVCache, x, slot, pos
     B = x.shape[0]
     mlb = cache.max_len if max_len_bound is None else int(max_len_bound)
     cs, ws_, cc = cfg.struct(), w.struct(), cache.struct()
-    nbytes = lib.decode_layer_workspace_size(C.byref(cs), B, min(mlb, cache.max_len))
+    nbytes = lib.decode_layer_workspace_size(C.byref(cs), B, _resolved_bound(cache, mlb))
     if workspace is None:
         workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=x.device)
     out = torch.empty_like(x) if out is None else _need(out, torch.float32, "out")
@@ -400,7 +416,7 @@ def prefill_layer(cfg: LayerConfig, w: LayerWeights, cache: KVCache, x, slot: in
     T = x.shape[0]
     mlb = cache.max_len if max_len_bound is None else int(max_len_bound)
     cs, ws_, cc = cfg.struct(), w.struct(), cache.struct()
-    nbytes = lib.prefill_layer_workspace_size(C.byref(cs), T, min(mlb, cache.max_len))
+    nbytes = lib.prefill_layer_workspace_size(C.byref(cs), T, _resolved_bound(cache, mlb))
     if workspace is None:
         workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=x.device)
     out = torch.empty_like(x) if out is None else _need(out, torch.float32, "out")
@@ -419,7 +435,7 @@ class DecodeLayerCall:
         self.B = x.shape[0]
         self.mlb = cache.max_len if max_len_bound is None else int(max_len_bound)
         self._cs, self._ws, self._cc = cfg.struct(), w.struct(), cache.struct()
-        nbytes = lib.decode_layer_workspace_size(C.byref(self._cs), self.B, min(self.mlb, cache.max_len))
+        nbytes = lib.decode_layer_workspace_size(C.byref(self._cs), self.B, _resolved_bound(cache, self.mlb))
         self.workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=x.device)
         self._keep = (cfg, w, cache, x, slot, pos, out)
         self._args = (C.byref(self._cs), C.byref(self._ws), C.byref(self._cc), _ptr(x), _ptr(slot), _ptr(pos), self.B,

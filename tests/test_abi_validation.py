@@ -106,3 +106,31 @@ def test_helpers_validation(L):
     assert L.inv_trace_events(events, 4) == INVALID
     assert L.inv_trace_events(None, 0) == OK
     assert L.inv_selftest_wait_timeout(0, None) == INVALID
+    assert L.inv_selftest_gemm_wait_timeout(PTR, 1 << 20, 0, None) == INVALID
+    assert L.inv_selftest_gemm_wait_timeout(None, 1 << 20, 1000, None) == INVALID
+    assert L.inv_selftest_gemm_wait_timeout(PTR, 1024, 1000, None) == WORKSPACE
+
+
+def test_workspace_sizes_use_the_resolved_bound(inv, L):
+    """A call with max_len_bound <= 0 resolves its bound to cache->max_len; the
+    size functions take that resolved bound and have no size for <= 0."""
+    Cfg = inv.LayerConfigStruct
+    good = Cfg(256, 8, 2, 128, 512, 512, 1e-6, 0.088)
+    assert L.attn_decode_workspace_size(4, 32, 0) == 0
+    assert L.decode_layer_workspace_size(C.byref(good), 4, 0) == 0
+    assert L.prefill_layer_workspace_size(C.byref(good), 4, -5) == 0
+    # a workspace sized with the cache's max_len is accepted by a call that passes bound 0
+    w = inv.LayerWeightsStruct(*([PTR.value] * 12))
+    c = cache(inv, hkv=2, max_len=512)
+    need = L.decode_layer_workspace_size(C.byref(good), 4, 512)
+    assert need > L.decode_layer_workspace_size(C.byref(good), 4, 256) > 0
+    assert L.decode_layer(C.byref(good), C.byref(w), C.byref(c), PTR, PTR, PTR, 4, 0, PTR2, PTR, need - 1,
+                          None) == WORKSPACE
+    a = L.attn_decode_fixedsplit
+    c8 = cache(inv, max_len=8192)
+    need_a = L.attn_decode_workspace_size(4, 32, 8192)
+    assert a(PTR, 4, 32, C.byref(c8), PTR, PTR, 0, 256, 0.1, PTR, None, None, PTR, need_a - 1, None) == WORKSPACE
+    # the no-alloc variant applies its size limit to the resolved bound too
+    c_big = cache(inv, max_len=8192)
+    assert L.attn_decode_fixedsplit_noalloc(PTR, 80, 32, C.byref(c_big), PTR, PTR, 0, 256, 0.1, PTR, None, None,
+                                            None) == WORKSPACE

@@ -99,7 +99,7 @@ def test_decode_layer_full_shape_batch_invariance(inv):
     x = torch.randn((n_seq, H), generator=g, device="cuda")
     pos = torch.full((n_seq,), ctx, dtype=torch.int32, device="cuda")
     ref_out = None
-    for B in (256, 128, 37, 8, 1):
+    for B in (256, 128, 37, 32, 8, 1):
         perm = torch.from_numpy(synth.permutation(n_seq, seed=B)).cuda()
         out = torch.empty_like(x)
         for a in range(0, n_seq, B):
@@ -136,6 +136,60 @@ def test_prefill_layer_matches_decode_layer_full_shape(inv):
         start += T
     assert torch.equal(a.k, b.k) and torch.equal(a.v, b.v)
     assert torch.equal(a.k_scale, b.k_scale) and torch.equal(a.v_scale, b.v_scale)
+    assert status() == inv.INV_OK
+
+
+def test_prefill_layer_full_shape_oracle_parity(inv):
+    """prefill_layer against the float64 oracle layer at the 7B-like shape: a
+    700-token prompt in chunks of 300, 77 and 323 rows, so chunk boundaries fall
+    inside 256-key splits and inside the attention's 64-row blocks.  Every row
+    of every chunk is within 1e-5 (normwise) of the oracle, and the cache the
+    GPU wrote gives decode_layer's bits for the next decoded token."""
+    p = host_layer(seed=110)
+    cfg, w = gpu_layer(inv, p, 1024)
+    oc = ref.KVCache.empty(1, HKV, 1024, D)
+    gc = inv.KVCache(n_slots=1, n_kv_heads=HKV, max_len=1024)
+    xs = synth.normal((701, H), seed=111)
+    start = 0
+    for T in (300, 77, 323):
+        x = xs[start:start + T]
+        y = inv.prefill_layer(cfg, w, gc, dev(x), 0, start)
+        want = ref.decode_layer(p, oc, x, np.zeros(T, np.int64), np.arange(start, start + T))
+        err = rowwise_err(host(y), want)
+        assert err.max() <= TOL, (start, err.max())
+        start += T
+    # one decoded token after the prompt, against the oracle too
+    y = inv.decode_layer(cfg, w, gc, dev(xs[700:701]), dev(np.zeros(1, np.int32)), dev(np.array([700], np.int32)))
+    want = ref.decode_layer(p, oc, xs[700:701], np.zeros(1, np.int64), np.array([700]))
+    assert rowwise_err(host(y), want).max() <= TOL
+    assert status() == inv.INV_OK
+
+
+def test_lm_head_logits_oracle_parity(inv):
+    """The stack head at the vocabulary size 32000: final RMSNorm (fused split)
+    and the compensated LM-head GEMM (N = 32000, 250 panels) against the
+    float64 oracle on the same hidden states, normwise 1e-5 per row, for a
+    ragged number of rows; each row's logits are bit-identical for every
+    batch size; greedy ids equal the oracle's argmax where its top-2 margin is
+    clear."""
+    V = 32000
+    x = synth.normal((133, H), seed=120)
+    g_final = synth.uniform(H, seed=121, lo=0.5, hi=1.5)
+    lm_head = synth.normal((H, V), seed=122, std=0.02)
+    P, e = inv.heal_pack_weight(dev(lm_head))
+    hi, lo = inv.rmsnorm_bi(dev(x), dev(g_final), 1e-6, want_y=False, want_split=True)
+    logits = inv.comp_gemm(hi, lo, P, e)
+    want = ref.rmsnorm(x, g_final, 1e-6) @ lm_head.astype(np.float64)
+    err = rowwise_err(host(logits), want)
+    assert err.max() <= TOL, err.max()
+    for M in (1, 8, 32, 128):
+        part = inv.comp_gemm(hi[:M].contiguous(), lo[:M].contiguous(), P, e)
+        assert torch.equal(part.view(torch.int32), logits[:M].view(torch.int32)), M
+    ids = host(inv.argmax_rows(logits))
+    srt = np.sort(want, axis=1)
+    clear = (srt[:, -1] - srt[:, -2]) > 1e-4 * np.abs(want).max(axis=1)
+    assert clear.sum() > 100
+    assert np.array_equal(ids[clear], ref.argmax_lowest(want)[clear])
     assert status() == inv.INV_OK
 
 
@@ -246,7 +300,7 @@ def test_stack_per_layer_divergence_from_oracle(inv):
     layers, embed, g_final, lm_head = _stack_params(n_layers, V, seed=400)
     prompt = synth.token_ids(T, V, seed=401)
     st = GpuStack(inv, layers, embed, g_final, lm_head, max_len=512)
-    hidden, ids, _ = st.forward(prompt, np.arange(T))
+    hidden, ids, gpu_logits = st.forward(prompt, np.arange(T))
     sp = ref.StackParams(embed=embed, layers=layers, g_final=g_final, lm_head=lm_head)
     caches = [ref.KVCache.empty(1, HKV, 512, D) for _ in range(n_layers)]
     logits, oids, ohidden = ref.stack_forward(sp, caches, prompt, np.zeros(T, np.int64), np.arange(T),
@@ -254,6 +308,9 @@ def test_stack_per_layer_divergence_from_oracle(inv):
     errs = [float(rowwise_err(host(hidden[l]), ohidden[l]).max()) for l in range(n_layers)]
     print("per-layer normwise divergence:", ["%.2e" % e for e in errs])
     assert max(errs) <= 2e-4, errs
+    # the head itself on the GPU's final hidden states: logits within 1e-5 of the oracle head
+    head_want = ref.rmsnorm(host(hidden[-1]), g_final, 1e-6) @ lm_head.astype(np.float64)
+    assert rowwise_err(host(gpu_logits), head_want).max() <= TOL
     srt = np.sort(logits, axis=1)
     clear = (srt[:, -1] - srt[:, -2]) > 1e-4 * np.abs(logits).max(axis=1)
     assert np.array_equal(host(ids)[clear], oids[clear])
@@ -306,29 +363,28 @@ def test_stack_32_layers_8192_prompt_chunked_prefill_and_128_decode_steps(inv):
     def run(chunked):
         caches = [inv.KVCache(n_slots=1, n_kv_heads=HKV, max_len=max_len) for _ in range(n_layers)]
         spans = [(a, min(T, a + chunk)) for a in range(0, T, chunk)] if chunked else [(0, T)]
-        last = None
+        # every layer's output for every prompt position (32 x 8192 x 4096 fp32 = 4.3 GB)
+        hidden = torch.empty((n_layers, T, H), dtype=torch.float32, device="cuda")
         for a, b in spans:
             x = inv.embed_gather(embed, prompt[a:b].contiguous())
             for l in range(n_layers):
-                x = inv.prefill_layer(cfg, layers[l], caches[l], x, 0, a)
-            last = x
-        ids = [int(head(last[-1:].contiguous())[0])]
-        dec_states = []
+                x = inv.prefill_layer(cfg, layers[l], caches[l], x, 0, a, out=hidden[l, a:b])
+        ids = [int(head(hidden[-1, -1:].contiguous())[0])]
+        dec_states = torch.empty((n_dec, n_layers, H), dtype=torch.float32, device="cuda")
         for t in range(n_dec):
             x = inv.embed_gather(embed, torch.tensor([ids[-1]], dtype=torch.int32, device="cuda"))
             for l in range(n_layers):
                 x = inv.decode_layer(cfg, layers[l], caches[l], x, torch.zeros(1, dtype=torch.int32, device="cuda"),
-                                     torch.tensor([T + t], dtype=torch.int32, device="cuda"))
-            dec_states.append(x[0].clone())
+                                     torch.tensor([T + t], dtype=torch.int32, device="cuda"), out=dec_states[t, l:l + 1])
             ids.append(int(head(x)[0]))
-        return caches, last, ids, torch.stack(dec_states)
+        return caches, hidden, ids, dec_states
 
-    c1, last1, ids1, dec1 = run(chunked=False)
-    c2, last2, ids2, dec2 = run(chunked=True)
+    c1, hid1, ids1, dec1 = run(chunked=False)
+    c2, hid2, ids2, dec2 = run(chunked=True)
     assert status() == inv.INV_OK
-    assert torch.equal(last1.view(torch.int32)[-chunk:], last2.view(torch.int32))  # final layer, last chunk
-    for l in range(n_layers):                                                     # every layer's cache
+    for l in range(n_layers):   # every layer's hidden states at every prompt position, and its cache
+        assert torch.equal(hid1[l].view(torch.int32), hid2[l].view(torch.int32)), l
         assert torch.equal(c1[l].k, c2[l].k) and torch.equal(c1[l].v, c2[l].v), l
         assert torch.equal(c1[l].k_scale, c2[l].k_scale) and torch.equal(c1[l].v_scale, c2[l].v_scale), l
     assert ids1 == ids2
-    assert torch.equal(dec1.view(torch.int32), dec2.view(torch.int32))
+    assert torch.equal(dec1.view(torch.int32), dec2.view(torch.int32))   # every layer, every decode step

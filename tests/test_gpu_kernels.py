@@ -72,10 +72,10 @@ def test_rmsnorm_parity(inv, hidden):
     y, hi, lo = inv.rmsnorm_bi(dev(x), dev(gamma), 1e-6, want_y=True, want_split=True)
     want = ref.rmsnorm(x, gamma, 1e-6)
     assert rowwise_err(host(y), want).max() <= 1e-6
-    # the fused split equals heal_split of the kernel's own fp32 output
-    h2, l2 = inv.heal_split(y)
-    assert torch.equal(hi.view(torch.int16), h2.view(torch.int16))
-    assert torch.equal(lo.view(torch.int16), l2.view(torch.int16))
+    # the fused split is the oracle's binary16 encoding of the kernel's own fp32 output, bit for bit
+    h_want, l_want, _ = enc.heal_split(host(y))
+    assert np.array_equal(bits16(hi), h_want)
+    assert np.array_equal(bits16(lo), l_want)
 
 
 def test_rmsnorm_rows_batch_invariant(inv):
@@ -268,8 +268,10 @@ def test_attention_parity_edges(inv, Hq, Hkv):
     want = ref.attention_decode(q, oc, slot, lens, sigma)
     err = rowwise_err(host(out).reshape(B * Hq, 128), want.reshape(B * Hq, 128))
     assert err.max() <= TOL, err.max()
-    h2, l2 = inv.heal_split(out.reshape(B * Hq, 128))
-    assert torch.equal(hi.reshape(B * Hq, 128).view(torch.int16), h2.view(torch.int16))
+    # the combine's fused split is the oracle's binary16 encoding of its fp32 output, bit for bit
+    h_want, l_want, _ = enc.heal_split(host(out).reshape(B * Hq, 128))
+    assert np.array_equal(bits16(hi).reshape(B * Hq, 128), h_want)
+    assert np.array_equal(bits16(lo).reshape(B * Hq, 128), l_want)
 
 
 def test_attention_config3_parity_and_composition(inv):
@@ -307,6 +309,18 @@ def test_bounded_wait_times_out_and_context_survives(inv):
     inv.inv_selftest_wait_timeout(2_000_000)  # 2 ms
     assert status() == inv.INV_ERR_TIMEOUT
     x = synth.normal((4, 64), seed=1)
+    hi, lo = inv.heal_split(dev(x))
+    assert np.array_equal(bits16(hi), enc.heal_split(x)[0])
+    assert status() == inv.INV_OK
+
+
+def test_gemm_consumer_wait_times_out_and_context_survives(inv):
+    """The down GEMM of a layer waits on the gate/up GEMM's tile counters; with
+    a counter that nothing completes, the wait must give up, record
+    INV_ERR_TIMEOUT and let the kernel exit with the context usable."""
+    inv.inv_selftest_gemm_wait_timeout(2_000_000)  # 2 ms
+    assert status() == inv.INV_ERR_TIMEOUT
+    x = synth.normal((4, 64), seed=2)
     hi, lo = inv.heal_split(dev(x))
     assert np.array_equal(bits16(hi), enc.heal_split(x)[0])
     assert status() == inv.INV_OK

@@ -47,16 +47,18 @@ def test_noalloc_matches_workspace_entry_point_twice(inv):
     slot, ld = dev(np.arange(B, dtype=np.int32)), dev(lens)
     sigma = float(np.float32(1 / np.sqrt(128)))
     want, want_hi, _ = inv.attn_decode_fixedsplit(q, cache, slot, ld, sigma, want_split=True)
-    first = inv.attn_decode_fixedsplit_noalloc(q, cache, slot, ld, sigma)
+    first, first_hi, _ = inv.attn_decode_fixedsplit_noalloc(q, cache, slot, ld, sigma, want_split=True)
     # a second, different call in between leaves other partials in the shared array
     q2 = q.flip(0).contiguous()
     inv.attn_decode_fixedsplit_noalloc(q2, cache, slot.flip(0).contiguous(), ld.flip(0).contiguous(), sigma)
     second, second_hi, _ = inv.attn_decode_fixedsplit_noalloc(q, cache, slot, ld, sigma, want_split=True)
     assert status() == inv.INV_OK
     w = host(want).reshape(B * Hq, 128).astype(np.float64)
-    for got in (first, second):
+    for got, got_hi in ((first, first_hi), (second, second_hi)):
         assert rowwise_err(host(got).reshape(B * Hq, 128), w).max() <= TOL
-    assert torch.equal(second_hi.view(torch.int16), want_hi.view(torch.int16))
+        # the same kernels run on the same inputs: the results are the same bits
+        assert torch.equal(got.view(torch.int32), want.view(torch.int32))
+        assert torch.equal(got_hi.view(torch.int16), want_hi.view(torch.int16))
 
 
 def test_noalloc_rejects_sizes_beyond_its_array(inv):
@@ -69,6 +71,10 @@ def test_noalloc_rejects_sizes_beyond_its_array(inv):
     ones = dev(np.ones(B, np.int32))
     with pytest.raises(inv.InvError) as ei:
         inv.attn_decode_fixedsplit_noalloc(q, cache, dev(np.zeros(B, np.int32)), ones, 0.1)
+    assert ei.value.code == inv.INV_ERR_WORKSPACE
+    # a bound <= 0 resolves to the cache's max_len, which does not fit either
+    with pytest.raises(inv.InvError) as ei:
+        inv.attn_decode_fixedsplit_noalloc(q, cache, dev(np.zeros(B, np.int32)), ones, 0.1, max_len_bound=0)
     assert ei.value.code == inv.INV_ERR_WORKSPACE
     # the same call with a smaller length bound fits and runs
     out = inv.attn_decode_fixedsplit_noalloc(q, cache, dev(np.zeros(B, np.int32)), ones, 0.1, max_len_bound=256)
