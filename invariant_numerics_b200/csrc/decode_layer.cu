@@ -115,12 +115,16 @@ int run_layer(const inv_layer_config* cfg, const inv_layer_weights* w, const inv
   // 2. qkv = h W_qkv
   INV_TRACED(1, inv::launch_comp_gemm(ws.h_hi, ws.h_lo, B, H, H, w->w_qkv, w->e_qkv, NQKV, ws.qkv, NQKV, nullptr, 0, s));
   // 3. rotary embedding of q and k; k, v -> INT16 cache; len = pos + 1
+  //    (it also clears the attention's split counters and the gate/up tile
+  //    counters of this layer; the previous layer has finished with them)
   INV_TRACED(2, inv::launch_rope_quant(ws.qkv, B, Hq, *cache, slot, pos, w->rope_cos, w->rope_sin, cfg->max_pos,
-                                       ws.q_rot, ws.lens, s));
-  // 4-5. fixed-split attention + ordered combine -> o hi/lo (kernels 3 and 4)
+                                       ws.q_rot, ws.lens, inv::attn_counters(ws.attn, B, Hq, mlb),
+                                       (int64_t)B * Hkv, ws.ready, (int64_t)(inv::gemm_ready_bytes(B, 2 * F) / 4), s));
+  // 4-5. fixed-split attention, the ascending fold of the splits inside it
+  //      (decode) or in a separate combine kernel (prefill) -> o hi/lo
   if (prefill_slot < 0) {
     INV_TRY(inv::launch_attention(ws.q_rot, B, Hq, *cache, slot, ws.lens, mlb, cfg->softmax_scale, ws.o, ws.o_hi,
-                                  ws.o_lo, ws.attn, s, 3));
+                                  ws.o_lo, ws.attn, s, 3, true));
   } else {
     INV_TRY(inv::launch_attention_prefill(ws.q_rot, B, Hq, *cache, prefill_slot, prefill_pos0, ws.lens, mlb,
                                           cfg->softmax_scale, ws.o, ws.o_hi, ws.o_lo, ws.attn, s, 3));
@@ -133,7 +137,6 @@ int run_layer(const inv_layer_config* cfg, const inv_layer_weights* w, const inv
   // 10. out = x1 + a W_down.  The down GEMM starts while the gate/up GEMM's
   // last tiles (a partial wave) run, loading each 64-column K block of a as
   // soon as the gate/up tile that stores it has published it.
-  if (cudaMemsetAsync(ws.ready, 0, inv::gemm_ready_bytes(B, 2 * F), s) != cudaSuccess) return INV_ERR_CUDA;
   INV_TRACED(7, inv::launch_comp_gemm_ex(ws.h2_hi, ws.h2_lo, B, H, H, w->w_gu, w->e_gu, 2 * F, nullptr, 0, nullptr, 0,
                                          ws.a_hi, ws.a_lo, F, ws.ready, nullptr, s));
   INV_TRACED(8, inv::launch_comp_gemm_ex(ws.a_hi, ws.a_lo, B, F, F, w->w_down, w->e_down, H, x_out, H, ws.x1, H,

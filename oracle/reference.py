@@ -208,6 +208,39 @@ def decode_layer(p: LayerParams, cache: KVCache, x, slot, pos, softmax_scale=Non
     return out
 
 
+def decode_layer_at(p: LayerParams, cache: KVCache, x, slot, pos, rows, softmax_scale=None):
+    """decode_layer evaluated at the chosen `rows` only.
+
+    The K/V of EVERY input row are computed (RMSNorm, the K and V projections,
+    rotary embedding of K) and quantised into the cache first, exactly as
+    decode_layer does; the query, attention, output projection and MLP are
+    then evaluated for the rows listed in `rows` alone.  Row r of the result
+    is decode_layer's row rows[r] (same float64 operations on the same values;
+    only the set of rows each product runs over differs).  Used for checks at
+    sampled positions of long prompts, where the whole layer at every position
+    would be too slow."""
+    x = f64(np.asarray(x, np.float32))
+    B = x.shape[0]
+    Hq, Hkv, D = p.n_heads, p.n_kv_heads, p.head_dim
+    sigma = np.float32(1.0 / np.sqrt(D)) if softmax_scale is None else np.float32(softmax_scale)
+    slot = np.asarray(slot, np.int64)
+    pos = np.asarray(pos, np.int64)
+    rows = np.asarray(rows, np.int64)
+
+    h = rmsnorm(x, p.g_attn, p.eps)
+    k = apply_rope((h @ f64(p.wk)).reshape(B, Hkv, D), pos, p.rope_base)
+    v = (h @ f64(p.wv)).reshape(B, Hkv, D)
+    cache.write("k", k.astype(np.float32), slot, pos)
+    cache.write("v", v.astype(np.float32), slot, pos)
+    n = len(rows)
+    q = apply_rope((h[rows] @ f64(p.wq)).reshape(n, Hq, D), pos[rows], p.rope_base)
+    o = attention_decode(q, cache, slot[rows], pos[rows] + 1, sigma).reshape(n, Hq * D)
+    x1 = x[rows] + o @ f64(p.wo)
+    h2 = rmsnorm(x1, p.g_mlp, p.eps)
+    a = silu(h2 @ f64(p.w_gate)) * (h2 @ f64(p.w_up))
+    return x1 + a @ f64(p.w_down)
+
+
 @dataclass
 class StackParams:
     embed: np.ndarray      # fp32 [V, H]

@@ -239,6 +239,27 @@ def test_decode_layer_prefill_matches_hf_llama_block():
     np.testing.assert_allclose(np.concatenate(parts), ours, rtol=1e-12, atol=1e-12)
 
 
+def test_decode_layer_at_sampled_rows_matches_full_layer():
+    """decode_layer_at (K/V of every row, the rest at chosen rows) gives the
+    full layer's rows and the same cache; pinned through decode_layer, which
+    the Hugging Face block pins above."""
+    H, F, T = 128, 256, 300
+    p = _small_layer(seed=4, H=H, F=F)
+    x = synth.normal((T, H), seed=5)
+    slot, pos = np.zeros(T, np.int64), np.arange(T)
+    c_full = ref.KVCache.empty(1, p.n_kv_heads, 320, p.head_dim)
+    c_at = ref.KVCache.empty(1, p.n_kv_heads, 320, p.head_dim)
+    full = ref.decode_layer(p, c_full, x, slot, pos)
+    rows = np.array([0, 1, 7, 255, 256, 299])
+    at = ref.decode_layer_at(p, c_at, x, slot, pos, rows)
+    np.testing.assert_allclose(at, full[rows], rtol=1e-12, atol=1e-12)
+    for a, b in ((c_full.k, c_at.k), (c_full.v, c_at.v), (c_full.ks, c_at.ks), (c_full.vs, c_at.vs)):
+        assert np.array_equal(a, b)
+    # a planted mistake (rows off by one) is caught
+    bad = ref.decode_layer_at(p, ref.KVCache.empty(1, p.n_kv_heads, 320, p.head_dim), x, slot, pos, rows + 1 - (rows == 299))
+    assert np.abs(bad - full[rows]).max() > 1e-3
+
+
 def test_decode_layer_zero_projections_is_identity():
     p = _small_layer(seed=3)
     p.wo[:] = 0
