@@ -47,11 +47,30 @@ H, HQ, HKV, D, F = 4096, 32, 8, 128, 11008
 BATCH, KV_LEN = 128, 2048
 REFERENCE_SECONDS = 60.0  # timed oracle work of the reference arm, at most
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) of one attn_split launch per decoded row at KV length
-# 2048, from an ncu capture of the kernel at B = 32 (273.22 MB read + 6.08 MB
-# written), scaled by rows.  Set to None whenever the kernel changes and the
-# capture has not been repeated.
-ATTN_SPLIT_DRAM_BYTES_PER_ROW_KV2048 = (273.222656e6 + 6.080512e6) / 32
+# DRAM traffic per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)
+# of the step's kernels, recorded by a capture of this benchmark's workload in
+# profiles/dram_traffic.txt together with the SHA-256 of the kernel's source
+# file at capture time: a record whose source has changed since is not used.
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+KERNEL_SOURCES = {"comp_gemm_kernel": "comp_gemm.cu", "attn_split_kernel": "attention.cu"}
+
+
+def captured_traffic(kernel: str, workload: str):
+    """(bytes per launch, note) from the capture record, or (None, why)."""
+    import hashlib
+    try:
+        with open(TRAFFIC_RECORD) as f:
+            rec = json.load(f).get(kernel)
+    except Exception:
+        return None, "no capture record"
+    if not rec or rec.get("workload") != workload:
+        return None, "no capture of this workload"
+    src = os.path.join(ROOT, "invariant_numerics_b200", "csrc", KERNEL_SOURCES[kernel])
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    if sha != rec.get("source_sha256"):
+        return None, "kernel source changed since the capture"
+    return rec["dram_bytes_per_launch"], rec.get("command", "")
 
 
 def load_peaks():
@@ -466,9 +485,8 @@ def run_ours(args, rank, world, local):
     st = inv.inv_get_device_status()
     if st != inv.INV_OK:
         raise RuntimeError(f"device status {inv.status_string(st)}")
-    # (decode_layer folds the attention splits inside the split kernel: no combine launch)
     kern_ms = {name: statistics.fmean(evs[k][2 * i].elapsed_time(evs[k][2 * i + 1]) for k in range(K))
-               for i, name in enumerate(inv.DECODE_LAYER_KERNEL_NAMES) if name != "attn_combine"}
+               for i, name in enumerate(inv.DECODE_LAYER_KERNEL_NAMES)}
 
     # ----- end to end through the C ABI with host buffers: every step uploads
     # its inputs from pinned host memory and downloads its output.  Two buffer
@@ -494,54 +512,80 @@ def run_ours(args, rank, world, local):
     with torch.cuda.graph(graphs[1]):
         call1()
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
-    up_done = [torch.cuda.Event() for _ in range(2)]
-    comp_done = [torch.cuda.Event() for _ in range(2)]
-    down_done = [torch.cuda.Event() for _ in range(2)]
-    barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    up.wait_event(e0)
-    down.wait_event(e0)
-    for k in range(K):
-        bi = k & 1
-        up.wait_event(comp_done[bi])        # step k-2 has finished reading this input set
-        with torch.cuda.stream(up):
-            xs[bi].copy_(x_host, non_blocking=True)
-            ss[bi].copy_(slot_host, non_blocking=True)
-            ps[bi].copy_(pos_host, non_blocking=True)
-            up_done[bi].record(up)
-        stream.wait_event(up_done[bi])
-        stream.wait_event(down_done[bi])    # step k-2's output has left this set
-        graphs[bi].replay()
-        comp_done[bi].record(stream)
-        down.wait_event(comp_done[bi])
-        with torch.cuda.stream(down):
-            y_hosts[bi].copy_(ys[bi], non_blocking=True)
-            down_done[bi].record(down)
-    stream.wait_event(down_done[0])
-    stream.wait_event(down_done[1])
-    e1.record(stream)
-    e1.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / K)
+    calls = [call, call1]
+
+    def e2e_run(step):
+        """K steps of `step(buffer set)` with every step's upload and download
+        inside the timed region; returns ms per step (max over ranks)."""
+        up_done = [torch.cuda.Event() for _ in range(2)]
+        comp_done = [torch.cuda.Event() for _ in range(2)]
+        down_done = [torch.cuda.Event() for _ in range(2)]
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        up.wait_event(e0)
+        down.wait_event(e0)
+        for k in range(K):
+            bi = k & 1
+            up.wait_event(comp_done[bi])        # step k-2 has finished reading this input set
+            with torch.cuda.stream(up):
+                xs[bi].copy_(x_host, non_blocking=True)
+                ss[bi].copy_(slot_host, non_blocking=True)
+                ps[bi].copy_(pos_host, non_blocking=True)
+                up_done[bi].record(up)
+            stream.wait_event(up_done[bi])
+            stream.wait_event(down_done[bi])    # step k-2's output has left this set
+            step(bi)
+            comp_done[bi].record(stream)
+            down.wait_event(comp_done[bi])
+            with torch.cuda.stream(down):
+                y_hosts[bi].copy_(ys[bi], non_blocking=True)
+                down_done[bi].record(down)
+        stream.wait_event(down_done[0])
+        stream.wait_event(down_done[1])
+        e1.record(stream)
+        e1.synchronize()
+        assert torch.equal(y_hosts[(K - 1) & 1], ys[(K - 1) & 1].cpu())
+        return max_over_ranks(e0.elapsed_time(e1) / K)
+
+    # the public call every step (host validation, tensor maps, launches), and
+    # the same call captured once as a CUDA graph and replayed
+    e2e_ms = e2e_run(lambda bi: calls[bi](stream))
+    e2e_graph_ms = e2e_run(lambda bi: graphs[bi].replay())
     h2d = x_host.numel() * 4 + slot_host.numel() * 4 + pos_host.numel() * 4
     d2h = y_hosts[0].numel() * 4
-    assert torch.equal(y_hosts[(K - 1) & 1], ys[(K - 1) & 1].cpu())
 
-    # ----- roofline of the dominant kernel (the attention split kernel)
+    # ----- rooflines: per kernel function, its share of the traced step; the
+    # largest is the line's `roofline`, the next `roofline_second`
     gemm_b, attn_b = layer_bytes(BATCH, KV_LEN)
     hbm = peaks["hbm_gbs"]
-    attn_gbs = attn_b / (kern_ms["attn_split"] * 1e-3) / 1e9
     kernels = {}
     for name, t in kern_ms.items():
         ent = {"us": round(t * 1e3, 2)}
-        if name in gemm_b:
-            ent["gbs"] = round(gemm_b[name] / (t * 1e-3) / 1e9, 1)
+        byts = gemm_b.get(name, attn_b if name == "attn_split" else None)
+        if byts is not None:
+            ent["algorithmic_bytes"] = byts
+            ent["gbs"] = round(byts / (t * 1e-3) / 1e9, 1)
             ent["frac_hbm"] = round(ent["gbs"] / hbm, 3)
-        if name == "attn_split":
-            ent["gbs"] = round(attn_gbs, 1)
-            ent["frac_hbm"] = round(attn_gbs / hbm, 3)
         kernels[name] = ent
+    traced_us = sum(kern_ms.values()) * 1e3
+    workload = f"decode_layer H{H} Hq{HQ} Hkv{HKV} D{D} F{F} B{BATCH} kv{KV_LEN}"
+
+    def roofline_of(kernel, names, byts_per_step):
+        us = sum(kern_ms[n] for n in names) * 1e3
+        launches = len(names)
+        achieved = byts_per_step / (us * 1e-6) / 1e9
+        traffic, src = captured_traffic(kernel, workload)
+        return {"kernel": kernel, "launches_per_step": launches, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                "traffic": round(traffic) if traffic is not None else None, "traffic_source": src,
+                "algorithmic_bytes_per_launch": round(byts_per_step / launches),
+                "us_per_launch": round(us / launches, 2), "share_of_traced_step": round(us / traced_us, 4),
+                "peak_source": f"{peak_kind} hbm_gbs"}
+    lines = sorted([roofline_of("comp_gemm_kernel", list(gemm_b), sum(gemm_b.values())),
+                    roofline_of("attn_split_kernel", ["attn_split"], attn_b)],
+                   key=lambda r: -r["share_of_traced_step"])
     step_bytes = sum(gemm_b.values()) + attn_b
     result = {
         "metric": "batch-invariant decode-layer tokens/s",
@@ -556,22 +600,21 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "f16 hi/lo products, f32 accumulate; int16 KV",
         "data": "synthetic",
-        "config": {"workload": f"decode_layer H{H} Hq{HQ} Hkv{HKV} D{D} F{F} B{BATCH} kv{KV_LEN}",
+        "config": {"workload": workload,
                    "global_batch": BATCH * world, "seq_len": KV_LEN, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (708.8 MB packed weights + 1.09 GB INT16 KV per step)"},
-        "roofline": {"kernel": "attn_split", "bound": "hbm", "achieved": round(attn_gbs, 1), "peak": hbm,
-                     "unit": "GB/s", "frac": round(attn_gbs / hbm, 4),
-                     "traffic": (round(ATTN_SPLIT_DRAM_BYTES_PER_ROW_KV2048 * BATCH)
-                                 if (KV_LEN == 2048 and ATTN_SPLIT_DRAM_BYTES_PER_ROW_KV2048) else None),
-                     "traffic_source": "ncu dram__bytes_read+write of a B=32 capture, scaled by rows",
-                     "peak_source": f"{peak_kind} hbm_gbs",
-                     "algorithmic_bytes_per_launch": attn_b},
+        "roofline": lines[0],
+        "roofline_second": lines[1],
         "step_roofline": {"bytes": step_bytes, "hbm_bound_ms": round(step_bytes / (hbm * 1e9) * 1e3, 4),
                           "frac": round(step_bytes / (hbm * 1e9) * 1e3 / ms, 4)},
         "kernels": kernels,
         "ms_per_step_without_graph": round(ms_traced, 4),
         "e2e": {"value": round(replicas.job_throughput(BATCH, world, e2e_ms), 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
+                "call": "decode_layer through the C ABI every step (host validation and launches inside the region)"},
+        "e2e_graph": {"value": round(replicas.job_throughput(BATCH, world, e2e_graph_ms), 1), "unit": "tokens/s",
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_graph_ms, 4),
+                      "call": "the same decode_layer call captured once in a CUDA graph, replayed every step"},
         "gpu_launches": K * len(kern_ms),
         "clocks": clocks,
         "wall_s_timed": round(t_wall, 3),
@@ -587,11 +630,20 @@ def run_ours(args, rank, world, local):
         # and the stack's divergence from it at the chunked-prefill size
         if not args.no_stack_divergence:
             result["stack_divergence"] = stack_divergence(inv, torch, device)
-        v, el, calls = time_oracle(args.oracle_rows, args.oracle_seconds)
+        v, el, ncalls = time_oracle(args.oracle_rows, args.oracle_seconds)
         result["cpu_baseline"] = {"value": round(v, 4), "unit": "tokens/s", "cores": cpu_cores_used(),
                                   "kind": "oracle",
-                                  "sample": f"{args.oracle_rows} sequences x {calls} oracle decode_layer calls "
+                                  "sample": f"{args.oracle_rows} sequences x {ncalls} oracle decode_layer calls "
                                             f"(same layer shape, kv {KV_LEN}), {el:.1f} s"}
+        try:
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                v1, el1, calls1 = time_oracle(args.oracle_rows, args.oracle_seconds / 2)
+            result["cpu_baseline"]["value_1thread"] = round(v1, 4)
+            result["cpu_baseline"]["sample_1thread"] = (f"{args.oracle_rows} sequences x {calls1} calls with the "
+                                                        f"BLAS pool limited to 1 thread, {el1:.1f} s")
+        except ImportError:
+            result["cpu_baseline"]["value_1thread"] = None
     replicas.barrier()
     del graph, graphs
     replicas.finalize()
@@ -664,7 +716,8 @@ def bench_components(inv, torch, device, peaks, peak_kind):
     gbs = byts / (t * 1e-3) / 1e9
     out["attention"] = {"B": B, "mean_len": float(lens.mean()), "us": round(t * 1e3, 2), "gbs": round(gbs, 1),
                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "bytes": byts,
-                        "note": "split + combine kernels, L2 flushed between launches"}
+                        "note": "one attn_decode_fixedsplit call (split kernel + ordered combine kernel), "
+                                "L2 flushed between launches"}
     assert inv.inv_get_device_status() == inv.INV_OK
     return out
 

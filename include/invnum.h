@@ -118,10 +118,9 @@ INV_API int inv_selftest_gemm_wait_timeout(void* workspace, size_t ws_bytes, lon
  * events != NULL and n_events >= 2 * INV_DECODE_LAYER_KERNELS, every later
  * decode_layer call records events[2i] before and events[2i+1] after its i-th
  * kernel launch, on the call's stream (i: 0 rmsnorm, 1 qkv GEMM, 2 rotary +
- * quantise, 3 attention splits, 4 attention combine -- recorded only by
- * prefill_layer, whose splits are folded by a separate kernel --, 5 output
- * GEMM, 6 rmsnorm, 7 gate/up GEMM with fused SwiGLU, 8 down GEMM).  events are
- * cudaEvent_t handles the caller created and keeps alive.  NULL / 0 switches tracing off.  Host-global.
+ * quantise, 3 attention splits, 4 attention combine, 5 output GEMM, 6 rmsnorm,
+ * 7 gate/up GEMM with fused SwiGLU, 8 down GEMM).  events are cudaEvent_t
+ * handles the caller created and keeps alive.  NULL / 0 switches tracing off.  Host-global.
  */
 #define INV_DECODE_LAYER_KERNELS 9
 INV_API int inv_trace_events(void** events, int n_events);
@@ -217,10 +216,7 @@ INV_API int kv_quant_int16(const float* x, int T, int64_t ld_x, const int32_t* s
  * dual-FP16 unpacked codes (code = 256 h + l, both exact in binary16) and the
  * hi/lo split of q, its own max, exp-sum and value sum; the splits are then
  * folded in ascending s.  Nothing depends on other rows or on len beyond the
- * row's own split count.  The fold runs in the CTA of the row's last split to
- * finish (a per-(row, kv head) arrival counter in the workspace decides which;
- * only that count is atomic, never a value), so the call is one kernel launch
- * after a memset of the counters.
+ * row's own split count.
  *   q        : fp32 [B][n_heads][128], 16-byte aligned.
  *   len      : int32 [B], 1 <= len[b] <= cache->max_len.
  *   max_len_bound : host upper bound on every len[b] (<= 0: cache->max_len);
@@ -251,8 +247,7 @@ INV_API int attn_decode_fixedsplit(const float* q, int B, int n_heads, const inv
  * synchronise the device).  No counterpart on the pages: it is an interface
  * variant only.  The split partials live in a file-scope device array of
  * INV_NOALLOC_SCRATCH_BYTES on every GPU that loads the library, held until
- * exit; each call clears the array's split counters (a memset on the call's
- * stream) before its kernel.  Calls needing more than that return INV_ERR_WORKSPACE and launch
+ * exit.  Calls needing more than that return INV_ERR_WORKSPACE and launch
  * nothing: the test is attn_decode_workspace_size(B, n_heads, L) >
  * INV_NOALLOC_SCRATCH_BYTES with the resolved bound L = min(max_len_bound,
  * cache->max_len), or L = cache->max_len when max_len_bound <= 0.  The first call on a device looks the array's address up
@@ -307,9 +302,8 @@ INV_API int rmsnorm_bi(const float* x, const float* gamma, int64_t rows, int hid
  *                 returns 0 for L <= 0).  Calls that overlap on the GPU need
  *                 separate workspaces.
  * Stream work: the layer's kernels only, all on `stream` (the rotary/quantise
- * kernel also clears the workspace counters the later kernels use).  The
- * attention folds its splits inside the split kernel (see
- * attn_decode_fixedsplit).  The W_down GEMM is launched as a
+ * kernel also clears the workspace's gate/up tile counters).  The W_down GEMM
+ * is launched as a
  * programmatic dependent of the gate/up GEMM and starts during its last
  * partial wave, loading each K block of a once the gate/up tile that stores it
  * has published it (no change to any product or sum).  All of this may be

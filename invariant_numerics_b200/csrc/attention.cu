@@ -52,7 +52,6 @@ struct __align__(1024) DecodeSmem {
   RowScratch rs;
   uint64_t bar_k, bar_v[4];    // V: one barrier per warp (its 64 keys)
   int abort;
-  int last;                    // this CTA is the last split of its (row, kv head) to finish
 };
 constexpr size_t kDecodeSmem = sizeof(DecodeSmem) + 1024;
 
@@ -390,90 +389,18 @@ __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& 
   if (kReuse) sync();  // the scratch and xo are reused by the next rows
 }
 
-// Fold the S split partials of one (row, head) in ascending split order (one
-// warp; lane l owns d = 4l .. 4l+3) and write o / l as fp32 and, if out_hi is
-// set, its binary16 hi/lo split.  L outside [1, len_limit] (a rejected row)
-// writes zeros.  Partials are read at L2 (ld.global.cg): in the fused form
-// they were written by other CTAs of the running grid.
-__device__ __forceinline__ void fold_splits(const float* __restrict__ po_rh, const float2* __restrict__ ml_rh, int L,
-                                            int len_limit, float* __restrict__ out_rh, __half* __restrict__ hi_rh,
-                                            __half* __restrict__ lo_rh, int lane, int* status) {
-  const float4* po = reinterpret_cast<const float4*>(po_rh) + lane;
-  float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (L >= 1 && L <= len_limit) {
-    const int S = (L + SPLIT - 1) / SPLIT;
-    float M = -INFINITY;  // exact max: order does not matter
-    for (int s0 = 0; s0 < S; s0 += 8) {
-      float2 v[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = s0 + j < S ? __ldcg(ml_rh + s0 + j) : make_float2(-INFINITY, 0.0f);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) M = fmaxf(M, v[j].x);
-    }
-    float l = 0.0f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0; s0 < S; s0 += 8) {  // splits folded in ascending order, 8 loads in flight
-      float2 v[8];
-      float4 o[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        v[j] = s0 + j < S ? __ldcg(ml_rh + s0 + j) : make_float2(-INFINITY, 0.0f);
-        o[j] = s0 + j < S ? __ldcg(po + (s0 + j) * 32) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (s0 + j >= S) break;
-        const float f = expf(__fsub_rn(v[j].x, M));
-        l = __fadd_rn(l, __fmul_rn(v[j].y, f));
-        acc.x = __fadd_rn(acc.x, __fmul_rn(o[j].x, f));
-        acc.y = __fadd_rn(acc.y, __fmul_rn(o[j].y, f));
-        acc.z = __fadd_rn(acc.z, __fmul_rn(o[j].z, f));
-        acc.w = __fadd_rn(acc.w, __fmul_rn(o[j].w, f));
-      }
-    }
-    res = make_float4(__fdiv_rn(acc.x, l), __fdiv_rn(acc.y, l), __fdiv_rn(acc.z, l), __fdiv_rn(acc.w, l));
-  }
-  reinterpret_cast<float4*>(out_rh)[lane] = res;
-  if (hi_rh) {
-    __half h[4], lo[4];
-    inv::split_hi_lo(res.x, h[0], lo[0]);
-    inv::split_hi_lo(res.y, h[1], lo[1]);
-    inv::split_hi_lo(res.z, h[2], lo[2]);
-    inv::split_hi_lo(res.w, h[3], lo[3]);
-    if (inv::f16_overflow(res.x) | inv::f16_overflow(res.y) | inv::f16_overflow(res.z) | inv::f16_overflow(res.w))
-      record_status(status, INV_ERR_RANGE);
-    uint2 hv, lv;
-    hv.x = pack_half2(h[0], h[1]);
-    hv.y = pack_half2(h[2], h[3]);
-    lv.x = pack_half2(lo[0], lo[1]);
-    lv.y = pack_half2(lo[2], lo[3]);
-    reinterpret_cast<uint2*>(hi_rh)[lane] = hv;
-    reinterpret_cast<uint2*>(lo_rh)[lane] = lv;
-  }
-}
-
-// Decode: one CTA per (row b, kv head h, split s).  Each CTA writes its
-// split's partials; the last of the row's S = ceil(L / 256) split CTAs of kv
-// head h to finish (a counter per (row, kv head), zero before the launch;
-// only the count is atomic, never a value) folds the S partials of each of
-// the G query heads in ascending split order and writes the output.
+// Decode: one CTA per (row b, kv head h, split s).
 __global__ void __launch_bounds__(THREADS, 3)
     attn_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const float* __restrict__ q, const float* __restrict__ kscale, const float* __restrict__ vscale,
                       const int32_t* __restrict__ slot, const int32_t* __restrict__ len, int Hq, int Hkv,
                       int n_slots, int max_len, int len_limit, int S_max, float sigma, float* __restrict__ part_o,
-                      float2* __restrict__ part_ml, int* __restrict__ counters, float* __restrict__ out,
-                      __half* __restrict__ out_hi, __half* __restrict__ out_lo, int* status, long long wait_ns) {
+                      float2* __restrict__ part_ml, int* status, long long wait_ns) {
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int G = Hq / Hkv;
   const int L = len[b], sl = slot[b];
   if (L < 1 || L > len_limit || sl < 0 || sl >= n_slots) {
     if (s == 0 && h == 0 && threadIdx.x == 0) record_status(status, INV_ERR_INVALID_ARG);
-    if (s == 0 && (threadIdx.x >> 5) < G) {  // a rejected row's output is zero
-      const int64_t rh = (int64_t)b * Hq + (int64_t)h * G + (threadIdx.x >> 5);
-      fold_splits(nullptr, nullptr, 0, len_limit, out + rh * 128, out_hi ? out_hi + rh * 128 : nullptr,
-                  out_lo ? out_lo + rh * 128 : nullptr, threadIdx.x & 31, status);
-    }
     return;
   }
   const int key0 = s * SPLIT;
@@ -537,24 +464,6 @@ __global__ void __launch_bounds__(THREADS, 3)
   // (only possible after a timed-out wait; immediate otherwise).
   if (tid == 0) inv::mbar_wait(&sm.bar_k, 0, wait_ns, nullptr, status);
   if (lane == 0 && v_issued) inv::mbar_wait(&sm.bar_v[tid >> 5], 0, wait_ns, nullptr, status);
-
-  // Publish this split; the last split of (b, h) to arrive folds them all.
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const int S = (L + SPLIT - 1) / SPLIT;
-    sm.last = atomicAdd(counters + (int64_t)b * Hkv + h, 1) == S - 1 ? 1 : 0;
-  }
-  __syncthreads();
-  if (sm.last) {
-    __threadfence();
-    const int warp = tid >> 5;
-    if (warp < G) {
-      const int64_t rh = obase + warp;
-      fold_splits(part_o + rh * S_max * 128, part_ml + rh * S_max, L, len_limit, out + rh * 128,
-                  out_hi ? out_hi + rh * 128 : nullptr, out_lo ? out_lo + rh * 128 : nullptr, lane, status);
-    }
-  }
 }
 
 // Prefill: rows r = 0..T-1 of one sequence (slot sl) at positions p0 + r.
@@ -633,8 +542,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   if (tid == 0) inv::mbar_wait(&sm.bar_kv, 0, wait_ns, nullptr, status);
 }
 
-// One warp per (row, head): fold splits s = 0, 1, ... in order (the prefill
-// form, whose split CTAs each cover a block of rows).
+// One warp per (row, head): fold splits s = 0, 1, ... in order.
 __global__ void attn_combine_kernel(const float* __restrict__ part_o, const float2* __restrict__ part_ml,
                                     const int32_t* __restrict__ len, int B, int Hq, int S_max, int len_limit,
                                     float* __restrict__ out, __half* __restrict__ out_hi, __half* __restrict__ out_lo,
@@ -643,8 +551,85 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o, const floa
   const int lane = threadIdx.x & 31;
   if (wid >= (int64_t)B * Hq) return;
   const int b = (int)(wid / Hq);
-  fold_splits(part_o + wid * S_max * 128, part_ml + wid * S_max, len[b], len_limit, out + wid * 128,
-              out_hi ? out_hi + wid * 128 : nullptr, out_lo ? out_lo + wid * 128 : nullptr, lane, status);
+  const float2* ml = part_ml + wid * S_max;
+  const float4* po = reinterpret_cast<const float4*>(part_o + wid * S_max * 128) + lane;
+  // The first 8 splits' (m, l) and o are requested together with len[b]: one
+  // memory round trip for KV lengths up to 2048.  Entries past the row's own
+  // split count are loaded (inside the partials buffer) but never used.
+  constexpr int PF = 8;
+  float2 v0[PF];
+  float4 o0[PF];
+#pragma unroll
+  for (int j = 0; j < PF; ++j) {
+    v0[j] = j < S_max ? ml[j] : make_float2(-INFINITY, 0.0f);
+    o0[j] = j < S_max ? po[j * 32] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const int L = len[b];
+  float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (L >= 1 && L <= len_limit) {
+    const int S = (L + SPLIT - 1) / SPLIT;
+    float M = -INFINITY;  // exact max: order does not matter
+#pragma unroll
+    for (int j = 0; j < PF; ++j)
+      if (j < S) M = fmaxf(M, v0[j].x);
+    for (int s0 = PF; s0 < S; s0 += 8) {
+      float2 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = s0 + j < S ? ml[s0 + j] : make_float2(-INFINITY, 0.0f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) M = fmaxf(M, v[j].x);
+    }
+    float l = 0.0f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    // splits folded in ascending order
+#pragma unroll
+    for (int j = 0; j < PF; ++j) {
+      if (j >= S) break;
+      const float f = expf(__fsub_rn(v0[j].x, M));
+      l = __fadd_rn(l, __fmul_rn(v0[j].y, f));
+      acc.x = __fadd_rn(acc.x, __fmul_rn(o0[j].x, f));
+      acc.y = __fadd_rn(acc.y, __fmul_rn(o0[j].y, f));
+      acc.z = __fadd_rn(acc.z, __fmul_rn(o0[j].z, f));
+      acc.w = __fadd_rn(acc.w, __fmul_rn(o0[j].w, f));
+    }
+    for (int s0 = PF; s0 < S; s0 += 8) {  // 8 loads in flight
+      float2 v[8];
+      float4 o[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        v[j] = s0 + j < S ? ml[s0 + j] : make_float2(-INFINITY, 0.0f);
+        o[j] = s0 + j < S ? po[(s0 + j) * 32] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (s0 + j >= S) break;
+        const float f = expf(__fsub_rn(v[j].x, M));
+        l = __fadd_rn(l, __fmul_rn(v[j].y, f));
+        acc.x = __fadd_rn(acc.x, __fmul_rn(o[j].x, f));
+        acc.y = __fadd_rn(acc.y, __fmul_rn(o[j].y, f));
+        acc.z = __fadd_rn(acc.z, __fmul_rn(o[j].z, f));
+        acc.w = __fadd_rn(acc.w, __fmul_rn(o[j].w, f));
+      }
+    }
+    res = make_float4(__fdiv_rn(acc.x, l), __fdiv_rn(acc.y, l), __fdiv_rn(acc.z, l), __fdiv_rn(acc.w, l));
+  }
+  reinterpret_cast<float4*>(out + wid * 128)[lane] = res;
+  if (out_hi) {
+    __half h[4], lo[4];
+    inv::split_hi_lo(res.x, h[0], lo[0]);
+    inv::split_hi_lo(res.y, h[1], lo[1]);
+    inv::split_hi_lo(res.z, h[2], lo[2]);
+    inv::split_hi_lo(res.w, h[3], lo[3]);
+    if (inv::f16_overflow(res.x) | inv::f16_overflow(res.y) | inv::f16_overflow(res.z) | inv::f16_overflow(res.w))
+      record_status(status, INV_ERR_RANGE);
+    uint2 hv, lv;
+    hv.x = pack_half2(h[0], h[1]);
+    hv.y = pack_half2(h[2], h[3]);
+    lv.x = pack_half2(lo[0], lo[1]);
+    lv.y = pack_half2(lo[2], lo[3]);
+    reinterpret_cast<uint2*>(out_hi + wid * 128)[lane] = hv;
+    reinterpret_cast<uint2*>(out_lo + wid * 128)[lane] = lv;
+  }
 }
 
 bool g_attn_attr[64] = {};
@@ -656,29 +641,19 @@ namespace inv {
 
 static int splits_for(int max_len_bound) { return (max_len_bound + SPLIT - 1) / SPLIT; }
 
-// [part_o: B Hq S 128 fp32][part_ml: B Hq S float2][split counters: B Hq int32]
-// (the counters use B Hkv <= B Hq of their room).
+// [part_o: B Hq S 128 fp32][part_ml: B Hq S float2]
 size_t attn_workspace_bytes(int B, int Hq, int max_len_bound) {
   const size_t S = (size_t)splits_for(max_len_bound);
-  return (size_t)B * Hq * S * (128 * sizeof(float) + sizeof(float2)) + (size_t)B * Hq * sizeof(int32_t);
-}
-
-int* attn_counters(void* ws, int B, int Hq, int max_len_bound) {
-  const size_t S = (size_t)splits_for(max_len_bound);
-  return reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + (size_t)B * Hq * S * (128 * sizeof(float) + sizeof(float2)));
+  return (size_t)B * Hq * S * (128 * sizeof(float) + sizeof(float2));
 }
 
 int launch_attention(const float* q, int B, int Hq, const inv_kv_cache& c, const int32_t* slot, const int32_t* len,
                      int max_len_bound, float sigma, float* out, uint16_t* out_hi, uint16_t* out_lo, void* ws,
-                     cudaStream_t s, int trace_base, bool counters_zeroed) {
+                     cudaStream_t s, int trace_base) {
   if (B == 0) return INV_OK;
   const int S_max = splits_for(max_len_bound);
   float* part_o = static_cast<float*>(ws);
   float2* part_ml = reinterpret_cast<float2*>(part_o + (size_t)B * Hq * S_max * 128);
-  int* counters = attn_counters(ws, B, Hq, max_len_bound);
-  if (!counters_zeroed &&
-      cudaMemsetAsync(counters, 0, (size_t)B * c.n_kv_heads * sizeof(int32_t), s) != cudaSuccess)
-    return INV_ERR_CUDA;
   const uint64_t rows = (uint64_t)c.n_slots * c.n_kv_heads * c.max_len;
   CUtensorMap tk, tv;
   int rc = make_tensor_map_2d(&tk, c.k, CU_TENSOR_MAP_DATA_TYPE_UINT16, 128, rows, 256, 64, 64,
@@ -696,12 +671,18 @@ int launch_attention(const float* q, int B, int Hq, const inv_kv_cache& c, const
   }
   dim3 grid(S_max, c.n_kv_heads, B);
   trace_record(2 * trace_base, s);
-  attn_split_kernel<<<grid, THREADS, kDecodeSmem, s>>>(
-      tk, tv, q, c.k_scale, c.v_scale, slot, len, Hq, c.n_kv_heads, c.n_slots, c.max_len, max_len_bound, S_max, sigma,
-      part_o, part_ml, counters, out, reinterpret_cast<__half*>(out_hi), reinterpret_cast<__half*>(out_lo),
-      status_ptr(), wait_limit_ns());
+  attn_split_kernel<<<grid, THREADS, kDecodeSmem, s>>>(tk, tv, q, c.k_scale, c.v_scale, slot, len, Hq, c.n_kv_heads,
+                                                     c.n_slots, c.max_len, max_len_bound, S_max, sigma, part_o, part_ml,
+                                                     status_ptr(), wait_limit_ns());
   INV_CHECK_LAUNCH();
   trace_record(2 * trace_base + 1, s);
+  const int64_t warps = (int64_t)B * Hq;
+  trace_record(2 * trace_base + 2, s);
+  attn_combine_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(
+      part_o, part_ml, len, B, Hq, S_max, max_len_bound, out, reinterpret_cast<__half*>(out_hi),
+      reinterpret_cast<__half*>(out_lo), status_ptr());
+  INV_CHECK_LAUNCH();
+  trace_record(2 * trace_base + 3, s);
   return INV_OK;
 }
 
@@ -777,7 +758,7 @@ int attn_decode_fixedsplit(const float* q, int B, int n_heads, const inv_kv_cach
   const int mlb = max_len_bound > 0 ? (max_len_bound < cache->max_len ? max_len_bound : cache->max_len) : cache->max_len;
   if (ws_bytes < inv::attn_workspace_bytes(B, n_heads, mlb)) return INV_ERR_WORKSPACE;
   return inv::launch_attention(q, B, n_heads, *cache, slot, len, mlb, softmax_scale, out, out_hi, out_lo, workspace,
-                               static_cast<cudaStream_t>(stream), -1, false);
+                               static_cast<cudaStream_t>(stream), -1);
 }
 
 }  // extern "C"

@@ -115,16 +115,14 @@ int run_layer(const inv_layer_config* cfg, const inv_layer_weights* w, const inv
   // 2. qkv = h W_qkv
   INV_TRACED(1, inv::launch_comp_gemm(ws.h_hi, ws.h_lo, B, H, H, w->w_qkv, w->e_qkv, NQKV, ws.qkv, NQKV, nullptr, 0, s));
   // 3. rotary embedding of q and k; k, v -> INT16 cache; len = pos + 1
-  //    (it also clears the attention's split counters and the gate/up tile
-  //    counters of this layer; the previous layer has finished with them)
+  //    (it also clears the gate/up tile counters of this layer; the previous
+  //    layer has finished with them)
   INV_TRACED(2, inv::launch_rope_quant(ws.qkv, B, Hq, *cache, slot, pos, w->rope_cos, w->rope_sin, cfg->max_pos,
-                                       ws.q_rot, ws.lens, inv::attn_counters(ws.attn, B, Hq, mlb),
-                                       (int64_t)B * Hkv, ws.ready, (int64_t)(inv::gemm_ready_bytes(B, 2 * F) / 4), s));
-  // 4-5. fixed-split attention, the ascending fold of the splits inside it
-  //      (decode) or in a separate combine kernel (prefill) -> o hi/lo
+                                       ws.q_rot, ws.lens, ws.ready, (int64_t)(inv::gemm_ready_bytes(B, 2 * F) / 4), s));
+  // 4-5. fixed-split attention + ordered combine -> o hi/lo (kernels 3 and 4)
   if (prefill_slot < 0) {
     INV_TRY(inv::launch_attention(ws.q_rot, B, Hq, *cache, slot, ws.lens, mlb, cfg->softmax_scale, ws.o, ws.o_hi,
-                                  ws.o_lo, ws.attn, s, 3, true));
+                                  ws.o_lo, ws.attn, s, 3));
   } else {
     INV_TRY(inv::launch_attention_prefill(ws.q_rot, B, Hq, *cache, prefill_slot, prefill_pos0, ws.lens, mlb,
                                           cfg->softmax_scale, ws.o, ws.o_hi, ws.o_lo, ws.attn, s, 3));

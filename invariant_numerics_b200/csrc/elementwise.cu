@@ -325,11 +325,10 @@ __global__ void rope_quant_kernel(const float* __restrict__ qkv, int T, int Hq, 
                                   const int32_t* __restrict__ slot, const int32_t* __restrict__ pos,
                                   const float* __restrict__ rope_cos, const float* __restrict__ rope_sin, int max_pos,
                                   float* __restrict__ q_out, int32_t* __restrict__ len_out, int* __restrict__ zero_a,
-                                  int64_t n_a, int* __restrict__ zero_b, int64_t n_b, int* status) {
+                                  int64_t n_a, int* status) {
   {
     const int64_t t0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x, stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = t0; i < n_a; i += stride) zero_a[i] = 0;
-    for (int64_t i = t0; i < n_b; i += stride) zero_b[i] = 0;
   }
   const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -438,14 +437,13 @@ int launch_rmsnorm(const float* x, const float* gamma, int64_t rows, int hidden,
 
 int launch_rope_quant(const float* qkv, int T, int Hq, const inv_kv_cache& c, const int32_t* slot,
                       const int32_t* pos, const float* rope_cos, const float* rope_sin, int max_pos, float* q_out,
-                      int32_t* len_out, int* zero_a, int64_t n_a, int* zero_b, int64_t n_b, cudaStream_t s) {
+                      int32_t* len_out, int* zero_a, int64_t n_a, cudaStream_t s) {
   if (T == 0) return INV_OK;
   const int64_t warps = (int64_t)T * (Hq + 2 * c.n_kv_heads);
   const int threads = 256;
   const int64_t blocks = (warps * 32 + threads - 1) / threads;
   rope_quant_kernel<<<(unsigned)blocks, threads, 0, s>>>(qkv, T, Hq, c, slot, pos, rope_cos, rope_sin, max_pos, q_out,
-                                                        len_out, zero_a, zero_a ? n_a : 0, zero_b, zero_b ? n_b : 0,
-                                                        status_ptr());
+                                                        len_out, zero_a, zero_a ? n_a : 0, status_ptr());
   INV_CHECK_LAUNCH();
   return INV_OK;
 }

@@ -12,11 +12,11 @@ namespace inv {
 int launch_rmsnorm(const float* x, const float* gamma, int64_t rows, int hidden, float eps, float* y,
                    uint16_t* yh, uint16_t* yl, cudaStream_t s);
 
-// Also sets zero_a[0 .. n_a) and zero_b[0 .. n_b) to zero (counters the
-// layer's later kernels need cleared; either may be null).
+// Also sets zero_a[0 .. n_a) to zero (counters a later kernel of the layer
+// needs cleared; may be null).
 int launch_rope_quant(const float* qkv, int T, int Hq, const inv_kv_cache& c, const int32_t* slot,
                       const int32_t* pos, const float* rope_cos, const float* rope_sin, int max_pos, float* q_out,
-                      int32_t* len_out, int* zero_a, int64_t n_a, int* zero_b, int64_t n_b, cudaStream_t s);
+                      int32_t* len_out, int* zero_a, int64_t n_a, cudaStream_t s);
 
 
 // Panel width (output columns per GEMM tile and per packed panel) of a weight
@@ -47,16 +47,13 @@ int launch_comp_gemm_ex(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, i
 inline size_t gemm_ready_bytes(int64_t M, int N) { return (size_t)((M + 127) / 128) * (size_t)(N / 128) * 4; }
 
 // Workspace layout of the attention: partial o and partial (m, l) per
-// (row, head, split), then one split counter per (row, kv head).
+// (row, head, split).
 size_t attn_workspace_bytes(int B, int Hq, int max_len_bound);
-int* attn_counters(void* ws, int B, int Hq, int max_len_bound);
-// Decode attention: split kernel with the ascending fold of each row's splits
-// done by the row's last split CTA.  counters_zeroed: the caller has already
-// cleared the B * n_kv_heads split counters on this stream (otherwise a
-// memset does).  trace_base < 0: no tracing.
+// Decode attention: split kernel, then the ascending fold of each row's
+// splits (combine kernel).  trace_base < 0: no tracing.
 int launch_attention(const float* q, int B, int Hq, const inv_kv_cache& c, const int32_t* slot, const int32_t* len,
                      int max_len_bound, float sigma, float* out, uint16_t* out_hi, uint16_t* out_lo, void* ws,
-                     cudaStream_t s, int trace_base, bool counters_zeroed);
+                     cudaStream_t s, int trace_base);
 
 // Prefill form: rows t = 0..T-1 are consecutive positions pos0 + t of the
 // sequence in `slot`; each split's K/V is loaded once for all rows that reach

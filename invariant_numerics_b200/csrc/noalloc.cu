@@ -14,9 +14,8 @@
 // device; make that first call before any stream capture.  Every call on a
 // device shares the one array and leaves the last call's partials in it:
 // calls whose kernels overlap on the GPU (different streams, no ordering)
-// race on it.  Of its contents only the per-(row, kv head) split counters must
-// start at zero; every call clears them with a memset on its stream before the
-// kernel (the partials are always written before they are read).
+// race on it.  Nothing in it needs clearing between calls -- the split kernel
+// writes every partial the combine kernel reads.
 #include <mutex>
 
 #include "common.cuh"
@@ -77,5 +76,5 @@ extern "C" int attn_decode_fixedsplit_noalloc(const float* q, int B, int n_heads
   const int rc = scratch_address(&scratch);
   if (rc != INV_OK) return rc;
   return inv::launch_attention(q, B, n_heads, *cache, slot, len, mlb, softmax_scale, out, out_hi, out_lo, scratch,
-                               static_cast<cudaStream_t>(stream), -1, false);
+                               static_cast<cudaStream_t>(stream), -1);
 }

@@ -55,8 +55,7 @@ def test_host_only_entry_points(lib):
     assert L.heal_packed_weight_bytes(0, 64) == 0
     L.attn_decode_workspace_size.restype = ctypes.c_size_t
     # (m, l) + o[128] per (row, head, split of 256)
-    # partials (128 fp32 o + (m, l)) per (row, head, split), then one int32 split counter per (row, head)
-    assert L.attn_decode_workspace_size(2, 32, 257) == 2 * 32 * 2 * (128 * 4 + 8) + 2 * 32 * 4
+    assert L.attn_decode_workspace_size(2, 32, 257) == 2 * 32 * 2 * (128 * 4 + 8)
 
 
 def test_binding_module_exposes_the_same_names():
