@@ -714,6 +714,20 @@ def bench_components(inv, torch, device, peaks, peak_kind):
     S = (lens.astype(np.int64) + 255) // 256
     byts = int(lens.astype(np.int64).sum()) * HKV * 520 + B * HQ * D * 4 * 2 + int(S.sum()) * HQ * (D + 2) * 4 * 2
     gbs = byts / (t * 1e-3) / 1e9
+    # LAMP variant on the same workload: time, recompute rate, distance from the plain call
+    lamp = {}
+    for tau in (0.01, 0.1, 1.0):
+        tl = timed(lambda: inv.attn_decode_lamp(q, cache, slot, lens_d, 0.08838834764831845, tau, out=o,
+                                                workspace=ws))
+        ol, rec = inv.attn_decode_lamp(q, cache, slot, lens_d, 0.08838834764831845, tau, want_recompute=True,
+                                       workspace=ws)
+        plain = inv.attn_decode_fixedsplit(q, cache, slot, lens_d, 0.08838834764831845, workspace=ws)
+        valid = torch.arange(rec.shape[2], device=device)[None, None, :] < lens_d[:, None, None]
+        rate = float(rec[valid.expand_as(rec)].float().mean())
+        dist = float(((ol - plain).abs().amax(-1) / plain.abs().amax(-1)).max())
+        lamp[f"tau{tau}"] = {"us": round(tl * 1e3, 2), "gbs": round(byts / (tl * 1e-3) / 1e9, 1),
+                             "recompute_rate": round(rate, 5), "max_normwise_distance_from_plain": dist}
+    out["attention_lamp"] = lamp
     out["attention"] = {"B": B, "mean_len": float(lens.mean()), "us": round(t * 1e3, 2), "gbs": round(gbs, 1),
                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "bytes": byts,
                         "note": "one attn_decode_fixedsplit call (split kernel + ordered combine kernel), "

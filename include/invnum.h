@@ -262,6 +262,41 @@ INV_API int attn_decode_fixedsplit_noalloc(const float* q, int B, int n_heads, c
                                            float softmax_scale, float* out, uint16_t* out_hi, uint16_t* out_lo,
                                            inv_stream stream);
 
+/*
+ * attn_decode_lamp -- attn_decode_fixedsplit with LAMP-style selective
+ * recompute of the scores (LAMP summary, gist.science: section "Fondement
+ * théorique", item 3, the softmax condition 2 z_j (1 - z_j) |y_j| > tau for
+ * recomputing a KQ product; section "Stratégie d'implémentation", evaluate in
+ * low precision, select, recompute the selected in high precision; the
+ * relaxed threshold of "Résultats expérimentaux", free of the softmax
+ * normalisation).  Opt-in precision variant; its results are NOT those of
+ * attn_decode_fixedsplit.  Per (row, query head, key j):
+ *   low precision : y_lo_j from binary16 accumulation of q16 . code_j, q16 =
+ *                   rn16(q): with code = 256 h + l, two binary16 accumulators
+ *                   a_h <- rn16(q16_d h + a_h), a_l <- rn16(q16_d (l/256) + a_l)
+ *                   over d = 0..127 in order (one rounding per multiply-add),
+ *                   then in fp32 y_lo = ((256 a_h + 256 a_l) s_K,j) sigma;
+ *   decision      : recompute iff y_lo_j is not finite or
+ *                   (2 fl32(exp(y_lo_j - m_s))) |y_lo_j| > tau (fp32), m_s the
+ *                   largest finite y_lo of the key's 256-key split -- an upper
+ *                   bound of the strict criterion, evaluated per split;
+ *   score         : recomputed keys take the full-precision score of
+ *                   attn_decode_fixedsplit, the others keep y_lo; the softmax,
+ *                   values and split fold are attn_decode_fixedsplit's.
+ * The decision depends only on the row's own keys and split boundaries, so the
+ * variant is batch-invariant like the plain call.
+ *   tau        : threshold (not NaN); tau < 0 recomputes every score.
+ *   recompute  : uint8 [B][n_heads][recompute_ld] or NULL; byte (b, h, j) of
+ *                every key j < len[b] is set to 1 if its score was recomputed,
+ *                else 0 (bytes past len[b] are not written).  recompute_ld >=
+ *                the resolved length bound.
+ *   other arguments and errors as attn_decode_fixedsplit (same workspace size).
+ */
+INV_API int attn_decode_lamp(const float* q, int B, int n_heads, const inv_kv_cache* cache, const int32_t* slot,
+                             const int32_t* len, int max_len_bound, int split, float softmax_scale, float tau,
+                             float* out, uint16_t* out_hi, uint16_t* out_lo, uint8_t* recompute,
+                             int64_t recompute_ld, void* workspace, size_t ws_bytes, inv_stream stream);
+
 /* ------------------------------------------------------------------------
  * rmsnorm_bi -- [BI] table row "RMSNorm": always the data-parallel strategy,
  * one CTA per row and one fixed reduction order per row:

@@ -42,6 +42,15 @@ struct RowScratch {
   float red_m[4][4];
   float red_l[4][4];
   float red_w[4][4];
+  float red_mlo[4][4];  // LAMP: per-warp max of the low-precision scores
+};
+
+// LAMP selective recompute (decode, one row per call; see attn_decode_lamp).
+struct LampArgs {
+  float tau;                 // recompute threshold
+  const float* q;            // fp32 q of the row's heads in shared memory, [head][128]
+  uint8_t* sel;              // recompute flags of head 0 of the group at this split's first key, or null
+  int64_t sel_head_stride;
 };
 
 struct __align__(1024) DecodeSmem {
@@ -153,11 +162,25 @@ struct RowSet {
 //          thread once its warp has finished reading K (a warp reads and later
 //          overwrites only the codes of its own 64 keys); the decode kernel
 //          loads that warp's V codes into the warp's K slot there.
-template <int R, bool kReuse, class Sync, class IssueV, class WaitV>
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// kLamp (R = 1 only): each score is also evaluated in low precision -- q16 .
+// code accumulated in binary16, one rounding per multiply-add, over d in
+// ascending order, the high and low code bytes in two accumulators -- and the
+// scores whose relaxed criterion 2 exp(y_lo - m_lo) |y_lo| exceeds tau (m_lo
+// the split's largest finite low-precision score; non-finite ones always)
+// keep the full-precision value; the others continue with y_lo.
+template <int R, bool kReuse, bool kLamp, class Sync, class IssueV, class WaitV>
 __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& rows, int G, uint32_t kbase,
                                            uint32_t vbase, const float* ks, const float* vs, RowScratch* rs,
                                            float* xo, float sigma, int64_t head_stride_o, int64_t head_stride_ml,
-                                           bool ok, int* status, IssueV issue_v, WaitV wait_v) {
+                                           bool ok, int* status, const LampArgs& lamp, IssueV issue_v,
+                                           WaitV wait_v) {
+  static_assert(!kLamp || R == 1, "the low-precision pass is per row");
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
   int n_max = 0;
 #pragma unroll
@@ -194,6 +217,8 @@ __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& 
   // ---------------------------------------------------------------- scores --
   float tsc[R][4][2];
   float mx[R];
+  float tlo[4][2];          // kLamp: low-precision scores of this thread's keys
+  float mlo = -INFINITY;    // kLamp: their largest finite value
 #pragma unroll
   for (int r = 0; r < R; ++r) mx[r] = -INFINITY;
 #pragma unroll
@@ -201,6 +226,40 @@ __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& 
     const int kb = warp * 64 + mt * 16;
 #pragma unroll
     for (int r = 0; r < R; ++r) tsc[r][mt][0] = tsc[r][mt][1] = -INFINITY;
+    if constexpr (kLamp) tlo[mt][0] = tlo[mt][1] = -INFINITY;
+    if constexpr (kLamp) {
+      if (ok && kb < n_max) {
+        // keys kb + g and kb + g + 8 of head c, side by side in one half2
+        __half2 ah = __float2half2_rn(0.0f), al = ah;
+        const float* qh = lamp.q + c * 128;
+#pragma unroll 2
+        for (int d0 = 0; d0 < 128; d0 += 8) {
+          const uint4 c1 = lds128(code_addr(kbase, kb + g, d0));
+          const uint4 c2 = lds128(code_addr(kbase, kb + g + 8, d0));
+          const uint32_t w1[4] = {c1.x, c1.y, c1.z, c1.w}, w2[4] = {c2.x, c2.y, c2.z, c2.w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t a = (w1[j >> 1] >> (16 * (j & 1))) & 0xFFFFu, b = (w2[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+            uint32_t hp, lp;
+            unpack_dual(a | (b << 16), hp, lp);
+            const __half2 q2 = __float2half2_rn(qh[d0 + j]);
+            ah = __hfma2(q2, *reinterpret_cast<const __half2*>(&hp), ah);
+            al = __hfma2(q2, *reinterpret_cast<const __half2*>(&lp), al);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int key = kb + g + 8 * i;
+          const float h = __half2float(i ? __high2half(ah) : __low2half(ah));
+          const float l = __half2float(i ? __high2half(al) : __low2half(al));
+          const float y = __fmul_rn(__fmul_rn(__fadd_rn(__fmul_rn(256.0f, h), __fmul_rn(256.0f, l)), ks[key]), sigma);
+          if (key < rows.n[0]) {
+            tlo[mt][i] = y;
+            if (isfinite(y)) mlo = fmaxf(mlo, y);
+          }
+        }
+      }
+    }
     if (ok && kb < n_max) {
       float acc[R][4];
 #pragma unroll
@@ -231,6 +290,33 @@ __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& 
           tsc[r][mt][i] = key < rows.n[r] ? t : -INFINITY;
           mx[r] = fmaxf(mx[r], tsc[r][mt][i]);
         }
+      }
+    }
+  }
+  if constexpr (kLamp) {
+    // the split's largest finite low-precision score of head c, then the
+    // recompute decision of every key
+    mlo = fmaxf(mlo, __shfl_xor_sync(0xffffffffu, mlo, 4));
+    mlo = fmaxf(mlo, __shfl_xor_sync(0xffffffffu, mlo, 8));
+    mlo = fmaxf(mlo, __shfl_xor_sync(0xffffffffu, mlo, 16));
+    if (g == 0) rs[0].red_mlo[warp][c] = mlo;
+    sync();
+    const float Mlo = fmaxf(fmaxf(rs[0].red_mlo[0][c], rs[0].red_mlo[1][c]),
+                            fmaxf(rs[0].red_mlo[2][c], rs[0].red_mlo[3][c]));
+    mx[0] = -INFINITY;
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int key = warp * 64 + mt * 16 + g + 8 * i;
+        if (ok && key < rows.n[0]) {
+          const float y = tlo[mt][i];
+          const bool sel =
+              !isfinite(y) || __fmul_rn(__fmul_rn(2.0f, expf(__fsub_rn(y, Mlo))), fabsf(y)) > lamp.tau;
+          if (!sel) tsc[0][mt][i] = y;
+          if (lamp.sel != nullptr && c < G) lamp.sel[c * lamp.sel_head_stride + key] = sel ? 1 : 0;
+        }
+        mx[0] = fmaxf(mx[0], tsc[0][mt][i]);
       }
     }
   }
@@ -389,13 +475,16 @@ __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& 
   if (kReuse) sync();  // the scratch and xo are reused by the next rows
 }
 
-// Decode: one CTA per (row b, kv head h, split s).
+// Decode: one CTA per (row b, kv head h, split s).  kLamp: the LAMP variant
+// (tau, and the recompute flags sel [B][Hq][sel_ld] or null).
+template <bool kLamp>
 __global__ void __launch_bounds__(THREADS, 3)
     attn_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const float* __restrict__ q, const float* __restrict__ kscale, const float* __restrict__ vscale,
                       const int32_t* __restrict__ slot, const int32_t* __restrict__ len, int Hq, int Hkv,
                       int n_slots, int max_len, int len_limit, int S_max, float sigma, float* __restrict__ part_o,
-                      float2* __restrict__ part_ml, int* status, long long wait_ns) {
+                      float2* __restrict__ part_ml, int* status, long long wait_ns, float tau, uint8_t* sel,
+                      int64_t sel_ld) {
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int G = Hq / Hkv;
   const int L = len[b], sl = slot[b];
@@ -443,9 +532,10 @@ __global__ void __launch_bounds__(THREADS, 3)
 
   bool v_issued = false;
   const RowSet<1> rows = {{sm.qs}, {n}, {part_o + (obase * S_max + s) * 128}, {part_ml + obase * S_max + s}};
-  split_rows<1, false>(
+  const LampArgs lamp = {tau, sm.qs, sel != nullptr ? sel + obase * sel_ld + key0 : nullptr, sel_ld};
+  split_rows<1, false, kLamp>(
       tid, []() { __syncthreads(); }, rows, G, cbase, cbase, sm.ks, sm.vs, &sm.rs,
-      reinterpret_cast<float*>(sm.codes), sigma, (int64_t)S_max * 128, (int64_t)S_max, ok, status,
+      reinterpret_cast<float*>(sm.codes), sigma, (int64_t)S_max * 128, (int64_t)S_max, ok, status, lamp,
       [&]() {  // this warp is done with its K codes: bring its V codes into the same slot
         const int warp = tid >> 5;
         if (lane == 0 && ok && warp < nbox) {
@@ -536,8 +626,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       rows.out_o[i] = part_o + (obase * S_max + s) * 128;
       rows.out_ml[i] = part_ml + obase * S_max + s;
     }
-    split_rows<PF_R, true>(gtid, group_sync, rows, G, kbase, vbase, sm.ks, sm.vs, sm.rs[grp], sm.xo[grp][0], sigma,
-                           (int64_t)S_max * 128, (int64_t)S_max, ok, status, []() {}, [](bool okv) { return okv; });
+    split_rows<PF_R, true, false>(gtid, group_sync, rows, G, kbase, vbase, sm.ks, sm.vs, sm.rs[grp], sm.xo[grp][0],
+                                  sigma, (int64_t)S_max * 128, (int64_t)S_max, ok, status, LampArgs{}, []() {},
+                                  [](bool okv) { return okv; });
   }
   if (tid == 0) inv::mbar_wait(&sm.bar_kv, 0, wait_ns, nullptr, status);
 }
@@ -632,7 +723,6 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o, const floa
   }
 }
 
-bool g_attn_attr[64] = {};
 bool g_prefill_attr[64] = {};
 
 }  // namespace
@@ -647,9 +737,13 @@ size_t attn_workspace_bytes(int B, int Hq, int max_len_bound) {
   return (size_t)B * Hq * S * (128 * sizeof(float) + sizeof(float2));
 }
 
-int launch_attention(const float* q, int B, int Hq, const inv_kv_cache& c, const int32_t* slot, const int32_t* len,
-                     int max_len_bound, float sigma, float* out, uint16_t* out_hi, uint16_t* out_lo, void* ws,
-                     cudaStream_t s, int trace_base) {
+// The decode split kernel (plain or LAMP), then the ordered combine.
+template <bool kLamp>
+static int launch_decode(const float* q, int B, int Hq, const inv_kv_cache& c, const int32_t* slot,
+                         const int32_t* len, int max_len_bound, float sigma, float* out, uint16_t* out_hi,
+                         uint16_t* out_lo, void* ws, cudaStream_t s, int trace_base, float tau, uint8_t* sel,
+                         int64_t sel_ld) {
+  static bool attr_set[64] = {};
   if (B == 0) return INV_OK;
   const int S_max = splits_for(max_len_bound);
   float* part_o = static_cast<float*>(ws);
@@ -663,17 +757,17 @@ int launch_attention(const float* q, int B, int Hq, const inv_kv_cache& c, const
   if (rc != INV_OK) return rc;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !g_attn_attr[dev]) {
-    if (cudaFuncSetAttribute(attn_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecodeSmem) !=
-        cudaSuccess)
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(attn_split_kernel<kLamp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kDecodeSmem) != cudaSuccess)
       return INV_ERR_CUDA;
-    g_attn_attr[dev] = true;
+    attr_set[dev] = true;
   }
   dim3 grid(S_max, c.n_kv_heads, B);
   trace_record(2 * trace_base, s);
-  attn_split_kernel<<<grid, THREADS, kDecodeSmem, s>>>(tk, tv, q, c.k_scale, c.v_scale, slot, len, Hq, c.n_kv_heads,
-                                                     c.n_slots, c.max_len, max_len_bound, S_max, sigma, part_o, part_ml,
-                                                     status_ptr(), wait_limit_ns());
+  attn_split_kernel<kLamp><<<grid, THREADS, kDecodeSmem, s>>>(
+      tk, tv, q, c.k_scale, c.v_scale, slot, len, Hq, c.n_kv_heads, c.n_slots, c.max_len, max_len_bound, S_max, sigma,
+      part_o, part_ml, status_ptr(), wait_limit_ns(), tau, sel, sel_ld);
   INV_CHECK_LAUNCH();
   trace_record(2 * trace_base + 1, s);
   const int64_t warps = (int64_t)B * Hq;
@@ -684,6 +778,13 @@ int launch_attention(const float* q, int B, int Hq, const inv_kv_cache& c, const
   INV_CHECK_LAUNCH();
   trace_record(2 * trace_base + 3, s);
   return INV_OK;
+}
+
+int launch_attention(const float* q, int B, int Hq, const inv_kv_cache& c, const int32_t* slot, const int32_t* len,
+                     int max_len_bound, float sigma, float* out, uint16_t* out_hi, uint16_t* out_lo, void* ws,
+                     cudaStream_t s, int trace_base) {
+  return launch_decode<false>(q, B, Hq, c, slot, len, max_len_bound, sigma, out, out_hi, out_lo, ws, s, trace_base,
+                              0.0f, nullptr, 0);
 }
 
 int launch_attention_prefill(const float* q, int T, int Hq, const inv_kv_cache& c, int slot, int pos0,
@@ -727,7 +828,52 @@ int launch_attention_prefill(const float* q, int T, int Hq, const inv_kv_cache& 
 
 }  // namespace inv
 
+namespace {
+
+// Host validation shared by the decode attention entry points; on success *mlb
+// is the resolved length bound.
+int validate_decode(const float* q, int B, int n_heads, const inv_kv_cache* cache, const int32_t* slot,
+                    const int32_t* len, int max_len_bound, int split, float* out, uint16_t* out_hi, uint16_t* out_lo,
+                    int* mlb) {
+  if (!cache || B < 0 || n_heads <= 0) return INV_ERR_INVALID_ARG;
+  if (split != INV_KV_SPLIT) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (cache->head_dim != INV_HEAD_DIM || cache->n_kv_heads <= 0 || n_heads % cache->n_kv_heads != 0)
+    return INV_ERR_UNSUPPORTED_SHAPE;
+  const int G = n_heads / cache->n_kv_heads;
+  if (G != 1 && G != 2 && G != 4) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (cache->max_len <= 0 || cache->max_len % 64 != 0 || cache->n_slots <= 0) return INV_ERR_INVALID_ARG;
+  if ((uint64_t)cache->n_slots * cache->n_kv_heads * cache->max_len >= (1ull << 31)) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (B > 65535) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (B > 0 && (!q || !slot || !len || !out || !cache->k || !cache->v || !cache->k_scale || !cache->v_scale))
+    return INV_ERR_INVALID_ARG;
+  if ((out_hi == nullptr) != (out_lo == nullptr)) return INV_ERR_INVALID_ARG;
+  if (B > 0 && (!inv::aligned16(q) || !inv::aligned16(cache->k) || !inv::aligned16(cache->v) || !inv::aligned16(out)))
+    return INV_ERR_INVALID_ARG;
+  if (out_hi && ((reinterpret_cast<uintptr_t>(out_hi) | reinterpret_cast<uintptr_t>(out_lo)) & 7u))
+    return INV_ERR_INVALID_ARG;
+  *mlb = max_len_bound > 0 ? (max_len_bound < cache->max_len ? max_len_bound : cache->max_len) : cache->max_len;
+  return INV_OK;
+}
+
+}  // namespace
+
 extern "C" {
+
+int attn_decode_lamp(const float* q, int B, int n_heads, const inv_kv_cache* cache, const int32_t* slot,
+                     const int32_t* len, int max_len_bound, int split, float softmax_scale, float tau, float* out,
+                     uint16_t* out_hi, uint16_t* out_lo, uint8_t* recompute, int64_t recompute_ld, void* workspace,
+                     size_t ws_bytes, inv_stream stream) {
+  int mlb = 0;
+  const int rc = validate_decode(q, B, n_heads, cache, slot, len, max_len_bound, split, out, out_hi, out_lo, &mlb);
+  if (rc != INV_OK) return rc;
+  if (tau != tau) return INV_ERR_INVALID_ARG;  // NaN
+  if (B == 0) return INV_OK;
+  if (recompute != nullptr && recompute_ld < mlb) return INV_ERR_INVALID_ARG;
+  if (!workspace || !inv::aligned16(workspace)) return INV_ERR_INVALID_ARG;
+  if (ws_bytes < inv::attn_workspace_bytes(B, n_heads, mlb)) return INV_ERR_WORKSPACE;
+  return inv::launch_decode<true>(q, B, n_heads, *cache, slot, len, mlb, softmax_scale, out, out_hi, out_lo, workspace,
+                                  static_cast<cudaStream_t>(stream), -1, tau, recompute, recompute_ld);
+}
 
 size_t attn_decode_workspace_size(int B, int n_heads, int max_len_bound) {
   if (B <= 0 || n_heads <= 0 || max_len_bound <= 0) return 0;

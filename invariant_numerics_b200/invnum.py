@@ -69,6 +69,8 @@ _SIGS = {
                                     _sz, _p]),
     "attn_decode_fixedsplit_noalloc": (_i, [_p, _i, _i, C.POINTER(KVCacheStruct), _p, _p, _i, _i, _f, _p, _p,
                                             _p, _p]),
+    "attn_decode_lamp": (_i, [_p, _i, _i, C.POINTER(KVCacheStruct), _p, _p, _i, _i, _f, _f, _p, _p, _p, _p, _i64,
+                              _p, _sz, _p]),
     "rmsnorm_bi": (_i, [_p, _p, _i64, _i, _f, _p, _p, _p, _p]),
     "decode_layer_workspace_size": (_sz, [C.POINTER(LayerConfigStruct), _i, _i]),
     "decode_layer": (_i, [C.POINTER(LayerConfigStruct), C.POINTER(LayerWeightsStruct), C.POINTER(KVCacheStruct),
@@ -261,6 +263,28 @@ def attn_decode_fixedsplit(q, cache: KVCache, slot, lens, softmax_scale, max_len
                                       float(softmax_scale), _ptr(out), _ptr(hi), _ptr(lo), _ptr(workspace),
                                       workspace.numel(), _stream(stream)))
     return (out, hi, lo) if want_split else out
+
+
+def attn_decode_lamp(q, cache: KVCache, slot, lens, softmax_scale, tau, max_len_bound=None, out=None,
+                     want_recompute=False, workspace=None, stream=None):
+    """LAMP selective-recompute variant of attn_decode_fixedsplit: q fp32
+    [B, Hq, 128] -> out fp32 [B, Hq, 128] (and, if want_recompute, the uint8
+    recompute flags [B, Hq, L] for L = the resolved length bound)."""
+    _need(q, torch.float32, "q"), _need(slot, torch.int32, "slot"), _need(lens, torch.int32, "lens")
+    B, Hq, D = q.shape
+    mlb = cache.max_len if max_len_bound is None else int(max_len_bound)
+    L = _resolved_bound(cache, mlb)
+    out = torch.empty_like(q) if out is None else _need(out, torch.float32, "out")
+    rec = torch.zeros((B, Hq, L), dtype=torch.uint8, device=q.device) if want_recompute else None
+    nbytes = lib.attn_decode_workspace_size(B, Hq, L)
+    if workspace is None:
+        workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=q.device)
+    cs = cache.struct()
+    _check("attn_decode_lamp",
+           lib.attn_decode_lamp(_ptr(q), B, Hq, C.byref(cs), _ptr(slot), _ptr(lens), mlb, KV_SPLIT,
+                                float(softmax_scale), float(tau), _ptr(out), None, None, _ptr(rec), L,
+                                _ptr(workspace), workspace.numel(), _stream(stream)))
+    return (out, rec) if want_recompute else out
 
 
 NOALLOC_SCRATCH_BYTES = 34 << 20

@@ -149,6 +149,138 @@ def attention_decode(q, cache: KVCache, slot, length, softmax_scale, return_prob
 
 
 # ----------------------------------------------------------------------------
+# LAMP-style selective recompute of the attention scores  [LAMP summary
+# ("LAMP", gist.science), section "Fondement théorique", item 3 (softmax: the l1
+# objective and the condition 2 z_j (1 - z_j) |y_j| > tau for recomputing the
+# KQ product y_j), section "Stratégie d'implémentation" (evaluate in low
+# precision, select from the low-precision result, recompute the selected
+# components in higher precision) and the relaxed relative-threshold variant of
+# "Résultats expérimentaux" (no dependence on the normalisation constant, for
+# single-pass softmax kernels)]
+# ----------------------------------------------------------------------------
+
+def softmax_l1_sensitivity(y) -> np.ndarray:
+    """2 z_j (1 - z_j) |y_j| with z = softmax(y): the l1 change of the softmax
+    output, to first order, per unit relative error in the score y_j."""
+    y = f64(y)
+    z = np.exp(y - y.max())
+    z = z / z.sum()
+    return 2.0 * z * (1.0 - z) * np.abs(y)
+
+
+def lamp_relaxed_criterion(y, split: int = 256) -> np.ndarray:
+    """The relaxed criterion 2 exp(y_j - m_s) |y_j|, m_s the largest score of
+    the fixed `split`-key block (absolute positions split*s ..) that holds key
+    j: no normalisation constant is needed, and since z_j <= exp(y_j - m_s)
+    and 1 - z_j <= 1 it bounds the strict 2 z_j (1 - z_j) |y_j| from above, so
+    it selects every score the strict rule selects (and some more)."""
+    y = f64(y)
+    out = np.empty_like(y)
+    for s0 in range(0, y.shape[-1], split):
+        ys = y[..., s0:s0 + split]
+        zh = np.exp(ys - ys.max(axis=-1, keepdims=True))
+        out[..., s0:s0 + split] = 2.0 * zh * np.abs(ys)
+    return out
+
+
+def lamp_low_precision_scores(q16_bits, codes, scales, softmax_scale) -> np.ndarray:
+    """Scores y_lo_j accumulated in binary16 (the low-precision evaluation).
+
+    With code = 256 h + l (h the signed high byte, l the low byte, both exact
+    in binary16 as h and l/256), two binary16 accumulators run over
+    d = 0, 1, ..., D-1 in order, each step one fused multiply-add rounded once
+    to binary16 (round half to even):
+        a_h <- rn16(q16_d h_jd + a_h),   a_l <- rn16(q16_d (l_jd / 256) + a_l)
+    (a sum that leaves the binary16 range becomes +-inf).  Then, in fp32 and in
+    this order, y_lo_j = ((256 a_h + 256 a_l) s_j) sigma.
+      q16_bits : uint16 [D] binary16 bits of the query head
+      codes    : int16 [L, D] INT16 codes of the keys;  scales : fp32 [L]
+    Returns fp32 [L]."""
+    q16 = enc.f16_bits_to_f64(np.asarray(q16_bits, np.uint16))
+    c = np.asarray(codes, np.int64)
+    h = (c >> 8).astype(np.float64)                 # arithmetic shift: the signed high byte
+    l = (c & 255).astype(np.float64) / 256.0
+    a_h = np.zeros(c.shape[0], np.float64)
+    a_l = np.zeros(c.shape[0], np.float64)
+    for d in range(c.shape[1]):                     # products and sums exact in float64
+        a_h = enc.f16_bits_to_f64(enc.rn16_bits(q16[d] * h[:, d] + a_h))
+        a_l = enc.f16_bits_to_f64(enc.rn16_bits(q16[d] * l[:, d] + a_l))
+    with np.errstate(invalid="ignore", over="ignore"):
+        t = np.float32(256.0) * a_h.astype(np.float32) + np.float32(256.0) * a_l.astype(np.float32)
+        return (t * np.asarray(scales, np.float32)) * np.float32(softmax_scale)
+
+
+def lamp_criterion_f32(y_lo, split: int = 256) -> np.ndarray:
+    """The relaxed criterion of fp32 low-precision scores y_lo [L] (keys at
+    absolute positions 0..L-1) evaluated in fp32:
+        zh = fl32(exp(y - m_s)),  c = (2 zh) |y|,
+    m_s the largest finite score of the key's 256-key block; +inf for a
+    non-finite score (always recomputed)."""
+    y = np.asarray(y_lo, np.float32)
+    c = np.full(y.shape, np.inf, np.float32)
+    for s0 in range(0, y.shape[-1], split):
+        ys = y[s0:s0 + split]
+        fin = np.isfinite(ys)
+        if not fin.any():
+            continue
+        m = ys[fin].max()
+        with np.errstate(invalid="ignore", over="ignore"):
+            zh = np.exp((ys - m).astype(np.float64)).astype(np.float32)
+            c[s0:s0 + split] = np.where(fin, (np.float32(2.0) * zh) * np.abs(ys), np.inf)
+    return c
+
+
+def lamp_select(y_lo, tau, split: int = 256) -> np.ndarray:
+    """The recompute decision: lamp_criterion_f32(y_lo) > tau (fp32)."""
+    return lamp_criterion_f32(y_lo, split) > np.float32(tau)
+
+
+def attention_decode_lamp(q, cache: KVCache, slot, length, softmax_scale, tau, split: int = 256,
+                          return_selection=False, select=None):
+    """Decode attention with LAMP selective recompute of the scores.
+
+    Every score is first evaluated in low precision (lamp_low_precision_scores:
+    binary16 accumulation of q16 . code, q16 = rn16(q)); the scores that
+    lamp_select picks are recomputed in full precision, y_j = sigma q . K~_j
+    (the definition, float64), the others keep y_lo.  The output is the
+    softmax of these mixed scores over all keys times V~ (as attention_decode).
+    With tau < 0 everything is recomputed (attention_decode itself).
+    `select`, if given, replaces the decision: select[b] is a boolean [Hq, L]
+    mask (for comparing other selection rules, or for evaluating a decision
+    taken elsewhere)."""
+    q32 = np.asarray(q, np.float32)
+    q = f64(q32)
+    q16_bits = enc.rn16_bits(q)
+    B, Hq, D = q.shape
+    Hkv = cache.k.shape[1]
+    G = Hq // Hkv
+    sigma = np.float32(softmax_scale)
+    out = np.zeros((B, Hq, D), np.float64)
+    selection = []
+    for b in range(B):
+        L = int(length[b])
+        s = int(slot[b])
+        Kt = enc.kv_dequant(cache.k[s, :, :L], cache.ks[s, :, :L])
+        Vt = enc.kv_dequant(cache.v[s, :, :L], cache.vs[s, :, :L])
+        sel_b = np.zeros((Hq, L), bool)
+        y = np.zeros((Hq, L), np.float64)
+        for h in range(Hq):
+            kh = h // G
+            y_lo = lamp_low_precision_scores(q16_bits[b, h], cache.k[s, kh, :L], cache.ks[s, kh, :L], sigma)
+            y_hi = float(sigma) * (Kt[kh] @ q[b, h])
+            sel = lamp_select(y_lo, tau, split) if select is None else np.asarray(select[b][h], bool)
+            sel_b[h] = sel
+            y[h] = np.where(sel, y_hi, y_lo.astype(np.float64))
+        y = y - y.max(axis=-1, keepdims=True)
+        p = np.exp(y)
+        p = p / p.sum(axis=-1, keepdims=True)
+        for h in range(Hq):
+            out[b, h] = p[h] @ Vt[h // G]
+        selection.append(sel_b)
+    return (out, selection) if return_selection else out
+
+
+# ----------------------------------------------------------------------------
 # decode layer and layer stack (LLaMA-style block: RMSNorm -> GQA attention with
 # rotary embedding over the INT16 cache -> residual -> RMSNorm -> SwiGLU MLP ->
 # residual)

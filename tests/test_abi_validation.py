@@ -134,3 +134,18 @@ def test_workspace_sizes_use_the_resolved_bound(inv, L):
     c_big = cache(inv, max_len=8192)
     assert L.attn_decode_fixedsplit_noalloc(PTR, 80, 32, C.byref(c_big), PTR, PTR, 0, 256, 0.1, PTR, None, None,
                                             None) == WORKSPACE
+
+
+def test_lamp_validation(inv, L):
+    a = L.attn_decode_lamp
+    c = cache(inv)
+    nan = float("nan")
+    assert a(PTR, 4, 32, C.byref(c), PTR, PTR, 256, 256, 0.1, nan, PTR, None, None, None, 0, PTR, 10 ** 9,
+             None) == INVALID                                                     # tau NaN
+    assert a(PTR, 4, 32, C.byref(c), PTR, PTR, 256, 128, 0.1, 0.1, PTR, None, None, None, 0, PTR, 10 ** 9,
+             None) == UNSUPPORTED                                                 # split
+    assert a(PTR, 4, 32, C.byref(c), PTR, PTR, 256, 256, 0.1, 0.1, PTR, None, None, PTR2, 100, PTR, 10 ** 9,
+             None) == INVALID                                                     # recompute_ld < bound
+    assert a(PTR, 4, 32, C.byref(c), PTR, PTR, 256, 256, 0.1, 0.1, PTR, None, None, None, 0, PTR, 16,
+             None) == WORKSPACE
+    assert a(PTR, 0, 32, C.byref(c), PTR, PTR, 256, 256, 0.1, 0.1, PTR, None, None, None, 0, None, 0, None) == OK

@@ -168,6 +168,145 @@ def test_attention_single_key_and_equal_keys():
         np.testing.assert_allclose(o5[0, h], Vd[0].mean(axis=0), rtol=1e-13, atol=1e-15)
 
 
+# ------------------------------------------------ LAMP selective recompute ----
+
+def _softmax(y):
+    e = np.exp(y - y.max())
+    return e / e.sum()
+
+
+def test_softmax_l1_sensitivity_matches_finite_differences():
+    """2 z_j (1 - z_j) |y_j| is the l1 change of softmax(y) per unit relative
+    error of y_j (the LAMP summary's softmax criterion): checked against a
+    central finite difference of the softmax itself."""
+    y = np.random.Generator(np.random.PCG64(3)).normal(size=12) * 3.0
+    sens = ref.softmax_l1_sensitivity(y)
+    eps = 1e-6
+    for j in range(len(y)):
+        up, dn = y.copy(), y.copy()
+        up[j] *= 1 + eps
+        dn[j] *= 1 - eps
+        fd = np.abs(_softmax(up) - _softmax(dn)).sum() / (2 * eps)
+        assert abs(fd - sens[j]) <= 1e-6 * max(sens.max(), 1e-12), (j, fd, sens[j])
+
+
+def test_lamp_relaxed_criterion_is_blockwise_and_bounds_the_strict_one():
+    y = np.random.Generator(np.random.PCG64(4)).normal(size=600) * 4.0
+    rel = ref.lamp_relaxed_criterion(y, 256)
+    # an upper bound of the strict criterion over the whole row (so it selects
+    # a superset), and the block maximum itself has the relaxed value 2 |y|
+    strict = ref.softmax_l1_sensitivity(y)
+    assert np.all(rel >= strict * (1 - 1e-12))
+    for s0 in (0, 256, 512):
+        j = s0 + int(np.argmax(y[s0:s0 + 256]))
+        assert rel[j] == 2.0 * abs(y[j])
+    # blocks sit at absolute positions: changing block 1 leaves block 0 alone
+    y2 = y.copy()
+    y2[300] += 50.0
+    rel2 = ref.lamp_relaxed_criterion(y2, 256)
+    assert np.array_equal(rel2[:256], rel[:256]) and not np.array_equal(rel2[256:512], rel[256:512])
+
+
+def test_lamp_binary16_accumulation_model():
+    """The low-precision scores are a sequential binary16 accumulation: exact
+    while every partial sum is representable, and stuck where an addend falls
+    below half an ulp of the running sum (round half to even)."""
+    D = 128
+    one = enc.rn16_bits(np.array([1.0]))[0]
+    # small integers: every partial sum exact -> y_lo = sigma s q . code exactly
+    q16 = enc.rn16_bits(np.arange(D, dtype=np.float64) % 7 - 3)
+    codes = ((np.arange(3 * D).reshape(3, D) % 11) - 5).astype(np.int16) * 256 + 3
+    s = np.array([0.5, 1.0, 2.0], np.float32)
+    y = ref.lamp_low_precision_scores(q16, codes, s, 1.0)
+    exact = (codes.astype(np.float64) @ enc.f16_bits_to_f64(q16)) * s
+    np.testing.assert_array_equal(y, exact.astype(np.float32))
+    # 2048 first, then 127 addends of 1: 2048 + 1 rounds back to 2048 (tie to even) every time
+    q16 = np.full(D, one, np.uint16)
+    q16[0] = enc.rn16_bits(np.array([32.0]))[0]
+    codes = np.full((1, D), 256, np.int16)          # h = 1, l = 0
+    codes[0, 0] = 64 * 256                          # h = 64: 32 x 64 = 2048
+    y = ref.lamp_low_precision_scores(q16, codes, np.array([1.0], np.float32), 1.0)
+    assert y[0] == np.float32(256.0 * 2048.0)       # exact would be 256 x 2175
+    # the low byte goes through its own accumulator as l / 256
+    codes = np.full((1, D), 3, np.int16)            # h = 0, l = 3
+    q16 = np.full(D, one, np.uint16)
+    y = ref.lamp_low_precision_scores(q16, codes, np.array([1.0], np.float32), 1.0)
+    assert y[0] == np.float32(3.0 * D)              # 128 x 3/256 = 1.5 exactly, x 256
+    # negative codes: the high byte is signed (-1 = 256 (-1) + 255)
+    codes = np.full((1, D), -1, np.int16)
+    q8 = np.zeros(D, np.uint16)
+    q8[:8] = one                                    # 8 terms: a_h = -8, a_l = 8 x 255/256, both exact
+    y = ref.lamp_low_precision_scores(q8, codes, np.array([1.0], np.float32), 1.0)
+    assert y[0] == np.float32(-8.0)
+
+
+def test_lamp_select_relaxed_criterion_in_fp32():
+    y = np.random.Generator(np.random.PCG64(5)).normal(size=600).astype(np.float32) * 4
+    c64 = ref.lamp_relaxed_criterion(y.astype(np.float64), 256)
+    for tau in (1e-3, 1e-1, 1.0):
+        sel = ref.lamp_select(y, tau)
+        far = np.abs(c64 - tau) > 1e-5 * tau
+        assert np.array_equal(sel[far], (c64 > tau)[far])
+    y[10] = np.inf                                   # a non-finite score is always recomputed
+    assert ref.lamp_select(y, 1e30)[10] and not ref.lamp_select(y, 1e30)[11]
+
+
+def _lamp_case(seed, B=3, Hq=8, Hkv=2, L=700, D=128, qscale=3.0):
+    k = synth.kv_tensor(B * L, Hkv, D, seed=seed, scale=synth.channel_scale(Hkv, D, seed=seed + 1))
+    v = synth.kv_tensor(B * L, Hkv, D, seed=seed + 2)
+    k = k.reshape(B, L, Hkv, D).transpose(0, 2, 1, 3).copy()
+    v = v.reshape(B, L, Hkv, D).transpose(0, 2, 1, 3).copy()
+    cache = _cache_with(k, v)
+    q = synth.normal((B, Hq, D), seed=seed + 3, std=qscale)
+    return cache, q, np.array([L, L - 123, 257])[:B]
+
+
+def test_lamp_attention_limits():
+    cache, q, lens = _lamp_case(20)
+    sigma = np.float32(1 / np.sqrt(128))
+    slots = np.arange(len(lens))
+    full = ref.attention_decode(q, cache, slots, lens, sigma)
+    # tau < 0 recomputes every score: the plain attention
+    np.testing.assert_allclose(ref.attention_decode_lamp(q, cache, slots, lens, sigma, tau=-1.0), full,
+                               rtol=1e-12, atol=1e-13)
+    # a selection given explicitly: all -> the plain attention; none -> visibly off
+    all_sel = [np.ones((q.shape[1], L), bool) for L in lens]
+    np.testing.assert_allclose(ref.attention_decode_lamp(q, cache, slots, lens, sigma, 0.0, select=all_sel), full,
+                               rtol=1e-12, atol=1e-13)
+    no_sel = [np.zeros((q.shape[1], L), bool) for L in lens]
+    assert np.abs(ref.attention_decode_lamp(q, cache, slots, lens, sigma, 0.0, select=no_sel) - full).max() > 1e-5
+
+
+def test_lamp_selection_beats_random_selection_and_is_monotone():
+    """The summary's findings restated on a synthetic case: recomputing the
+    scores the criterion selects reduces the error of the binary16-accumulated
+    softmax, a random selection of as many scores does much less, and a higher
+    threshold selects fewer scores."""
+    cache, q, lens = _lamp_case(30)
+    sigma = np.float32(1 / np.sqrt(128))
+    slots = np.arange(len(lens))
+    full = ref.attention_decode(q, cache, slots, lens, sigma)
+    err = lambda o: float(np.abs(o - full).max(axis=-1).mean())
+    no_sel = [np.zeros((q.shape[1], L), bool) for L in lens]
+    e_none = err(ref.attention_decode_lamp(q, cache, slots, lens, sigma, 0.0, select=no_sel))
+    counts = []
+    for tau in (1e-2, 1e-1, 1.0):
+        out, sel = ref.attention_decode_lamp(q, cache, slots, lens, sigma, tau=tau, return_selection=True)
+        n = sum(int(s.sum()) for s in sel)
+        counts.append(n)
+        g = np.random.Generator(np.random.PCG64(int(tau * 1e4)))
+        rnd = []
+        for s in sel:
+            m = np.zeros(s.size, bool)
+            m[g.choice(s.size, int(s.sum()), replace=False)] = True
+            rnd.append(m.reshape(s.shape))
+        e_lamp = err(out)
+        e_rand = err(ref.attention_decode_lamp(q, cache, slots, lens, sigma, 0.0, select=rnd))
+        assert 0 < n < 0.25 * sum(s.size for s in sel)
+        assert e_lamp < 0.5 * e_rand and e_lamp < 0.5 * e_none, (tau, n, e_lamp, e_rand, e_none)
+    assert counts[0] >= counts[1] >= counts[2]
+
+
 # ---------------------------------------------------- layer and stack --------
 
 def _small_layer(seed=0, H=128, Hq=4, Hkv=2, D=32, F=256):
