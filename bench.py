@@ -73,14 +73,40 @@ def captured_traffic(kernel: str, workload: str):
     return rec["dram_bytes_per_launch"], rec.get("command", "")
 
 
+def _numeric_leaves(obj, path=()):
+    if isinstance(obj, dict):
+        for k, v in obj.items():
+            yield from _numeric_leaves(v, path + (str(k).lower(),))
+    elif isinstance(obj, (int, float)) and not isinstance(obj, bool):
+        yield "/".join(path), float(obj)
+
+
 def load_peaks():
+    """Measured peaks of this GPU model (HBM copy GB/s, dense bf16 TFLOP/s as
+    a burst and sustained), read from MEASURED_PEAKS.json at the repository
+    root whatever its nesting: each figure is the first numeric entry whose
+    key path names it.  A figure the file lacks (or a missing file) takes the
+    fallback value, and the returned kind says which."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
-            p = json.load(f)
-        return p, "measured"
+            leaves = list(_numeric_leaves(json.load(f)))
     except Exception:
-        return PEAKS_FALLBACK, "fallback"
+        return dict(PEAKS_FALLBACK), "fallback"
+    want = {
+        "hbm_gbs": lambda k: "hbm" in k and ("gbs" in k or "gb/s" in k or "gb_s" in k),
+        "bf16_tflops": lambda k: "bf16" in k and "tflop" in k and "sustain" not in k,
+        "bf16_tflops_sustained": lambda k: "bf16" in k and "tflop" in k and "sustain" in k,
+    }
+    peaks, found = {}, []
+    for name, match in want.items():
+        hit = next((v for k, v in leaves if match(k) and v > 0), None)
+        peaks[name] = hit if hit is not None else PEAKS_FALLBACK[name]
+        if hit is not None:
+            found.append(name)
+    if len(found) == len(want):
+        return peaks, "measured"
+    return peaks, "measured " + ",".join(found) + "; fallback for the rest" if found else "fallback"
 
 
 # ------------------------------------------------------------------ clocks --
