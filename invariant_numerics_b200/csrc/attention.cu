@@ -56,6 +56,7 @@ struct LampArgs {
 struct __align__(1024) DecodeSmem {
   uint8_t codes[CODE_BYTES];   // K codes, then V codes, then the warp exchange of O
   float qs[4 * 128];           // q of the row's G query heads (bulk copy with K)
+  uint32_t qfrag[512];         // their hi/lo MMA fragments
   float ks[SPLIT];
   float vs[SPLIT];
   RowScratch rs;
@@ -177,7 +178,8 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 template <int R, bool kReuse, bool kLamp, class Sync, class IssueV, class WaitV>
 __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& rows, int G, uint32_t kbase,
                                            uint32_t vbase, const float* ks, const float* vs, RowScratch* rs,
-                                           float* xo, float sigma, int64_t head_stride_o, int64_t head_stride_ml,
+                                           float* xo, uint32_t* qfrag, float sigma, int64_t head_stride_o,
+                                           int64_t head_stride_ml,
                                            bool ok, int* status, const LampArgs& lamp, IssueV issue_v,
                                            WaitV wait_v) {
   static_assert(!kLamp || R == 1, "the low-precision pass is per row");
@@ -187,31 +189,42 @@ __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& 
   for (int r = 0; r < R; ++r) n_max = max(n_max, rows.n[r]);
 
   // B fragments of S^T = K Q^T: column g is query head g/2 of the group, its
-  // hi part for even g and lo part for odd g; rows k = d.
+  // hi part for even g and lo part for odd g; rows k = d.  Every warp needs
+  // the same fragments, so the group splits each q value once: pair p =
+  // (row r, k-step ks, i, head, c) holds d = 16 ks + 2 c + 8 i and d + 1, and
+  // its hi and lo words go to lanes 4 (2 head) + c and 4 (2 head + 1) + c at
+  // qfrag[((r 4 + j) 32 + lane) 4 + e] for ks 2 + i = 4 j + e, so that each
+  // lane then reads its 16 words as 4 conflict-free 128-bit loads.
   uint32_t qf[R][8][2];
   {
-    const int head = g >> 1;
-    const bool lo = (g & 1) != 0;
     bool bad = false;
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
+    for (int k = 0; k < 2 * R; ++k) {
+      const int r = k >> 1, rem = (tid + THREADS * k) & 255;
+      const int cc = rem & 3, head = (rem >> 2) & 3, q16 = rem >> 4;  // q16 = ks 2 + i
+      const int d = 16 * (q16 >> 1) + 2 * cc + 8 * (q16 & 1);
       const bool valid = head < G && rows.n[r] > 0;
-      const float* qh = rows.q[r] + head * 128;
-#pragma unroll
-      for (int ks_ = 0; ks_ < 8; ++ks_) {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int d = 16 * ks_ + 2 * c + 8 * i;
-          const float x0 = valid ? qh[d] : 0.0f, x1 = valid ? qh[d + 1] : 0.0f;
-          __half h0, l0, h1, l1;
-          inv::split_hi_lo(x0, h0, l0);
-          inv::split_hi_lo(x1, h1, l1);
-          bad |= inv::f16_overflow(x0) | inv::f16_overflow(x1);
-          qf[r][ks_][i] = lo ? pack_half2(l0, l1) : pack_half2(h0, h1);
-        }
-      }
+      const float2 x = valid ? *reinterpret_cast<const float2*>(rows.q[r] + head * 128 + d) : make_float2(0.f, 0.f);
+      __half h0, l0, h1, l1;
+      inv::split_hi_lo(x.x, h0, l0);
+      inv::split_hi_lo(x.y, h1, l1);
+      bad |= inv::f16_overflow(x.x) | inv::f16_overflow(x.y);
+      uint32_t* dst = qfrag + ((r * 4 + (q16 >> 2)) * 32 + 8 * head + cc) * 4 + (q16 & 3);
+      dst[0] = pack_half2(h0, h1);
+      dst[16] = pack_half2(l0, l1);  // lane + 4
     }
     if (bad) record_status(status, INV_ERR_RANGE);
+    sync();
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 w4 = lds128(inv::smem_u32(qfrag + ((r * 4 + j) * 32 + lane) * 4));
+        qf[r][2 * j][0] = w4.x;
+        qf[r][2 * j][1] = w4.y;
+        qf[r][2 * j + 1][0] = w4.z;
+        qf[r][2 * j + 1][1] = w4.w;
+      }
   }
 
   // ---------------------------------------------------------------- scores --
@@ -535,7 +548,7 @@ __global__ void __launch_bounds__(THREADS, 3)
   const LampArgs lamp = {tau, sm.qs, sel != nullptr ? sel + obase * sel_ld + key0 : nullptr, sel_ld};
   split_rows<1, false, kLamp>(
       tid, []() { __syncthreads(); }, rows, G, cbase, cbase, sm.ks, sm.vs, &sm.rs,
-      reinterpret_cast<float*>(sm.codes), sigma, (int64_t)S_max * 128, (int64_t)S_max, ok, status, lamp,
+      reinterpret_cast<float*>(sm.codes), sm.qfrag, sigma, (int64_t)S_max * 128, (int64_t)S_max, ok, status, lamp,
       [&]() {  // this warp is done with its K codes: bring its V codes into the same slot
         const int warp = tid >> 5;
         if (lane == 0 && ok && warp < nbox) {
@@ -626,7 +639,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       rows.out_o[i] = part_o + (obase * S_max + s) * 128;
       rows.out_ml[i] = part_ml + obase * S_max + s;
     }
+    // the q fragments of the rows use the start of the group's exchange buffer,
+    // which is written only after the last V read
     split_rows<PF_R, true, false>(gtid, group_sync, rows, G, kbase, vbase, sm.ks, sm.vs, sm.rs[grp], sm.xo[grp][0],
+                                  reinterpret_cast<uint32_t*>(sm.xo[grp][0]),
                                   sigma, (int64_t)S_max * 128, (int64_t)S_max, ok, status, LampArgs{}, []() {},
                                   [](bool okv) { return okv; });
   }
@@ -763,8 +779,8 @@ static int launch_decode(const float* q, int B, int Hq, const inv_kv_cache& c, c
       return INV_ERR_CUDA;
     attr_set[dev] = true;
   }
-  dim3 grid(S_max, c.n_kv_heads, B);
   trace_record(2 * trace_base, s);
+  dim3 grid(S_max, c.n_kv_heads, B);
   attn_split_kernel<kLamp><<<grid, THREADS, kDecodeSmem, s>>>(
       tk, tv, q, c.k_scale, c.v_scale, slot, len, Hq, c.n_kv_heads, c.n_slots, c.max_len, max_len_bound, S_max, sigma,
       part_o, part_ml, status_ptr(), wait_limit_ns(), tau, sel, sel_ld);
