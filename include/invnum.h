@@ -56,7 +56,9 @@ typedef enum {
   INV_ERR_WORKSPACE = 3,         /* workspace or output buffer smaller than required */
   INV_ERR_CUDA = 4,              /* a CUDA runtime/driver call failed */
   INV_ERR_RANGE = 5,             /* a value outside the binary16 range (|x| >= 65520) was split */
-  INV_ERR_TIMEOUT = 6            /* a bounded wait inside a kernel expired */
+  INV_ERR_TIMEOUT = 6,           /* a bounded wait inside a kernel expired */
+  INV_ERR_BOUNDS = 7             /* a kernel computed an index outside the buffer its caller
+                                    passed (recorded by the INV_DEBUG_BOUNDS build only) */
 } inv_status;
 
 /* Fixed algorithm constants (part of the numerics; not tunable). */
@@ -112,6 +114,28 @@ INV_API int inv_selftest_wait_timeout(long long wait_ns, inv_stream stream);
 #define INV_SELFTEST_GEMM_WS_BYTES 40192u
 INV_API int inv_selftest_gemm_wait_timeout(void* workspace, size_t ws_bytes, long long wait_ns,
                                            inv_stream stream);
+
+/*
+ * Index checks.  A library built with -DINV_DEBUG_BOUNDS (build option
+ * --debug-bounds, file libinvnum_debug.so) checks, in every kernel, each
+ * global-memory index it computes -- or, for a contiguous or strided block it
+ * accesses as a whole (a TMA tile, a split's scales, a row's partials), the
+ * block's first and last index -- against the extent of the buffer the
+ * caller passed, as stated by that call's contract.  An index outside it
+ * records INV_ERR_BOUNDS in the status word and the access is skipped (a
+ * block is skipped whole, before any of its loads is issued).  The normal
+ * build compiles the checks out.
+ * inv_debug_bounds_enabled: 1 in the checking build, 0 otherwise.
+ * inv_selftest_bounds: self-test of the check itself.  A kernel stores the
+ * value i to buf[i] for i = 0 .. n_written-1 while declaring the extent
+ * n_declared <= n_written (buf must hold n_declared floats): the stores
+ * i >= n_declared fail the check, are skipped and INV_ERR_BOUNDS is recorded.
+ * Errors: INV_ERR_UNSUPPORTED_SHAPE in the normal build (nothing launched, as
+ * the unchecked stores would leave the buffer); INV_ERR_INVALID_ARG for a null
+ * buf, n_declared < 0 or n_written < n_declared.
+ */
+INV_API int inv_debug_bounds_enabled(void);
+INV_API int inv_selftest_bounds(float* buf, int n_declared, int n_written, inv_stream stream);
 
 /*
  * Kernel tracing for decode_layer (profiling aid; off by default).  With

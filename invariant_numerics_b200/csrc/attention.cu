@@ -510,6 +510,20 @@ __global__ void __launch_bounds__(THREADS, 3)
   const int n = min(SPLIT, L - key0);
   const int nbox = (n + 63) >> 6;
   const int row0 = (int)(((int64_t)sl * Hkv + h) * max_len + key0);
+  const int64_t obase = (int64_t)b * Hq + (int64_t)h * G;
+  {
+    // index checks: the split's scales, the row's G query heads, their partials
+    // (part_o [B][Hq][S_max][128], part_ml [B][Hq][S_max]) and recompute flags
+    [[maybe_unused]] const int64_t BHq = (int64_t)gridDim.z * Hq;
+    if (!INV_SPAN_IN_BOUNDS(status, row0, row0 + n - 1, (int64_t)n_slots * Hkv * max_len) ||
+        !INV_SPAN_IN_BOUNDS(status, obase * 128, (obase + G) * 128 - 1, BHq * 128) ||
+        !INV_SPAN_IN_BOUNDS(status, (obase * S_max + s) * 128, ((obase + G - 1) * S_max + s) * 128 + 127,
+                            BHq * S_max * 128) ||
+        !INV_SPAN_IN_BOUNDS(status, obase * S_max + s, (obase + G - 1) * S_max + s, BHq * S_max) ||
+        (sel != nullptr &&
+         !INV_SPAN_IN_BOUNDS(status, obase * sel_ld + key0, (obase + G - 1) * sel_ld + key0 + n - 1, BHq * sel_ld)))
+      return;
+  }
 
   extern __shared__ uint8_t smem_raw[];
   DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -523,7 +537,6 @@ __global__ void __launch_bounds__(THREADS, 3)
     inv::fence_mbar_init();
   }
   __syncthreads();
-  const int64_t obase = (int64_t)b * Hq + (int64_t)h * G;
   if (tid == 0) {
     // q travels with K, so the scores start as soon as the codes land
     inv::mbar_arrive_expect_tx(&sm.bar_k, nbox * 2 * BOX_BYTES + G * 128 * 4);
@@ -582,7 +595,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                               const float* __restrict__ q, const float* __restrict__ kscale,
                               const float* __restrict__ vscale, int sl, int p0, int T, int Hq, int Hkv, int max_len,
                               int S_max, float sigma, float* __restrict__ part_o, float2* __restrict__ part_ml,
-                              int* status, long long wait_ns) {
+                              int* status, long long wait_ns, int n_slots) {
   const int s = blockIdx.x, h = blockIdx.y, rb = blockIdx.z;
   const int G = Hq / Hkv;
   const int key0 = s * SPLIT;
@@ -593,6 +606,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   const int n_max = min(SPLIT, p0 + r_last + 1 - key0);
   const int nbox = (n_max + 63) >> 6;
   const int row0 = (int)(((int64_t)sl * Hkv + h) * max_len + key0);
+  // index check of the split's scales (the rows' q and partials: per row below)
+  if (!INV_SPAN_IN_BOUNDS(status, row0, row0 + n_max - 1, (int64_t)n_slots * Hkv * max_len)) return;
 
   extern __shared__ uint8_t smem_raw[];
   PrefillSmem& sm = *reinterpret_cast<PrefillSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -638,6 +653,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       rows.n[i] = r0 + i <= r_last ? min(SPLIT, p0 + r + 1 - key0) : 0;
       rows.out_o[i] = part_o + (obase * S_max + s) * 128;
       rows.out_ml[i] = part_ml + obase * S_max + s;
+      // index checks of the row's q heads and partials; a failing row is left out
+      if (rows.n[i] > 0 &&
+          (!INV_SPAN_IN_BOUNDS(status, obase * 128, (obase + G) * 128 - 1, (int64_t)T * Hq * 128) ||
+           !INV_SPAN_IN_BOUNDS(status, (obase * S_max + s) * 128, ((obase + G - 1) * S_max + s) * 128 + 127,
+                               (int64_t)T * Hq * S_max * 128) ||
+           !INV_SPAN_IN_BOUNDS(status, obase * S_max + s, (obase + G - 1) * S_max + s, (int64_t)T * Hq * S_max)))
+        rows.n[i] = 0;
     }
     // the q fragments of the rows use the start of the group's exchange buffer,
     // which is written only after the last V read
@@ -657,6 +679,11 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o, const floa
   const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (wid >= (int64_t)B * Hq) return;
+  // index checks: the warp reads its S_max partials and writes one 128-wide row
+  if (!INV_SPAN_IN_BOUNDS(status, wid * S_max, wid * S_max + S_max - 1, (int64_t)B * Hq * S_max) ||
+      !INV_SPAN_IN_BOUNDS(status, wid * S_max * 128, (wid * S_max + S_max) * 128 - 1, (int64_t)B * Hq * S_max * 128) ||
+      !INV_SPAN_IN_BOUNDS(status, wid * 128, wid * 128 + 127, (int64_t)B * Hq * 128))
+    return;
   const int b = (int)(wid / Hq);
   const float2* ml = part_ml + wid * S_max;
   const float4* po = reinterpret_cast<const float4*>(part_o + wid * S_max * 128) + lane;
@@ -829,7 +856,7 @@ int launch_attention_prefill(const float* q, int T, int Hq, const inv_kv_cache& 
   trace_record(2 * trace_base, s);
   attn_prefill_split_kernel<<<grid, PF_THREADS, kPrefillSmem, s>>>(tk, tv, q, c.k_scale, c.v_scale, slot, pos0, T, Hq,
                                                                 c.n_kv_heads, c.max_len, S_max, sigma, part_o,
-                                                                part_ml, status_ptr(), wait_limit_ns());
+                                                                part_ml, status_ptr(), wait_limit_ns(), c.n_slots);
   INV_CHECK_LAUNCH();
   trace_record(2 * trace_base + 1, s);
   const int64_t warps = (int64_t)T * Hq;

@@ -46,6 +46,30 @@ __device__ __forceinline__ void record_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);  // first error wins
 }
 
+// Index checks of the INV_DEBUG_BOUNDS build: INV_IN_BOUNDS(status, i, n) is
+// true when 0 <= i < n, else it records INV_ERR_BOUNDS and is false;
+// INV_SPAN_IN_BOUNDS(status, first, last, n) checks a block accessed as a
+// whole by its first and last index.  The normal build compiles both to true
+// without evaluating the arguments.
+#ifdef INV_DEBUG_BOUNDS
+#define INV_IN_BOUNDS(status, i, n) ::inv::in_bounds((status), (int64_t)(i), (int64_t)(n))
+#define INV_SPAN_IN_BOUNDS(status, first, last, n) \
+  ::inv::span_in_bounds((status), (int64_t)(first), (int64_t)(last), (int64_t)(n))
+#else
+#define INV_IN_BOUNDS(status, i, n) true
+#define INV_SPAN_IN_BOUNDS(status, first, last, n) true
+#endif
+__device__ __forceinline__ bool in_bounds(int* status, int64_t i, int64_t n) {
+  if (i >= 0 && i < n) return true;
+  record_status(status, INV_ERR_BOUNDS);
+  return false;
+}
+__device__ __forceinline__ bool span_in_bounds(int* status, int64_t first, int64_t last, int64_t n) {
+  if (first >= 0 && first <= last && last < n) return true;
+  record_status(status, INV_ERR_BOUNDS);
+  return false;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -166,7 +166,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int kb = 0; kb < nkb; ++kb) {
           if (!inv::mbar_wait(&sm.empty[stage], phase ^ 1u, wait_ns, abort_flag, status)) goto producer_done;
           if (ready_in != nullptr && kb >= ready_upto &&
-              !wait_published(ready_in + (int64_t)mt * nkb, kb, nkb, &ready_upto, wait_ns, abort_flag, status))
+              (!INV_SPAN_IN_BOUNDS(status, (int64_t)mt * nkb, (int64_t)mt * nkb + nkb - 1, (int64_t)tiles_m * nkb) ||
+               !wait_published(ready_in + (int64_t)mt * nkb, kb, nkb, &ready_upto, wait_ns, abort_flag, status)))
             goto producer_done;
           uint8_t* st = sm.ring + stage * (2 * a_stride + W_BYTES);
           inv::mbar_arrive_expect_tx(&sm.full[stage], 2 * a_bytes + W_BYTES);
@@ -269,6 +270,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int c = 0; c < (EPI_COLS % 32 == 0 ? EPI_COLS : 0); c += 32) {
             const int f0 = (col0 + c) / 2;
+            // index checks: 32 column exponents, 16 outputs of gate_hi/lo [M][ld_g] (N / 2 used)
+            if (!INV_SPAN_IN_BOUNDS(status, col0 + c, col0 + c + 31, N) ||
+                !INV_SPAN_IN_BOUNDS(status, (int64_t)row * ld_g + f0, (int64_t)row * ld_g + f0 + 15,
+                                    (int64_t)(M - 1) * ld_g + N / 2))
+              continue;
             float v[32];
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
@@ -301,7 +307,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             gl[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
             gl[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
           }
-        } else if (row < M) {
+        } else if (row < M &&
+                   INV_SPAN_IN_BOUNDS(status, col0, col0 + EPI_COLS - 1, N) &&
+                   INV_SPAN_IN_BOUNDS(status, (int64_t)row * ld_y + col0, (int64_t)row * ld_y + col0 + EPI_COLS - 1,
+                                      (int64_t)(M - 1) * ld_y + N) &&
+                   (residual == nullptr ||
+                    INV_SPAN_IN_BOUNDS(status, (int64_t)row * ld_r + col0, (int64_t)row * ld_r + col0 + EPI_COLS - 1,
+                                       (int64_t)(M - 1) * ld_r + N))) {
+          // (index checks above: column exponents, y [M][ld_y] and residual [M][ld_r], N columns used)
           float* yr = y + (int64_t)row * ld_y + col0;
           const float* rr = residual ? residual + (int64_t)row * ld_r + col0 : nullptr;
 #pragma unroll
@@ -330,7 +343,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         // warp; the tile is complete when all EPI_WARPS warps have added
         __threadfence();
         __syncwarp();
-        if (lane == 0) inv::red_release_gpu_add(ready_out + (int64_t)mt * (N / BN) + nt, 1);
+        if (lane == 0 && INV_IN_BOUNDS(status, (int64_t)mt * (N / BN) + nt, (int64_t)tiles_m * (N / BN)))
+          inv::red_release_gpu_add(ready_out + (int64_t)mt * (N / BN) + nt, 1);
       }
     }
   epi_done:;

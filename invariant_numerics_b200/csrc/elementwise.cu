@@ -19,20 +19,20 @@ __global__ void heal_split_kernel(const float* __restrict__ x, int64_t rows, int
                                   int* status) {
   const int64_t c4 = (cols + 3) / 4;
   const int64_t total = rows * c4;
+  [[maybe_unused]] const int64_t n_x = (rows - 1) * ld_x + cols, n_out = (rows - 1) * ld_out + cols;  // extents
   bool bad = false;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = i / c4;
     const int64_t c = (i - r * c4) * 4;
-    const float* xr = x + r * ld_x;
-    __half* hr = hi + r * ld_out;
-    __half* lr = lo + r * ld_out;
     for (int j = 0; j < 4 && c + j < cols; ++j) {
-      const float v = xr[c + j];
+      const int64_t ix = r * ld_x + c + j, io = r * ld_out + c + j;
+      if (!INV_IN_BOUNDS(status, ix, n_x) || !INV_IN_BOUNDS(status, io, n_out)) continue;
+      const float v = x[ix];
       __half h, l;
       split_hi_lo(v, h, l);
       bad |= inv::f16_overflow(v);
-      hr[c + j] = h;
-      lr[c + j] = l;
+      hi[io] = h;
+      lo[io] = l;
     }
   }
   if (bad) record_status(status, INV_ERR_RANGE);
@@ -42,10 +42,12 @@ __global__ void heal_split_kernel(const float* __restrict__ x, int64_t rows, int
 __global__ void heal_split_vec_kernel(const float4* __restrict__ x, int64_t rows, int64_t c4, int64_t ld4,
                                       uint2* __restrict__ hi, uint2* __restrict__ lo, int64_t ldo4, int* status) {
   const int64_t total = rows * c4;
+  [[maybe_unused]] const int64_t n_x = (rows - 1) * ld4 + c4, n_out = (rows - 1) * ldo4 + c4;  // in float4s
   bool bad = false;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = i / c4;
     const int64_t c = i - r * c4;
+    if (!INV_IN_BOUNDS(status, r * ld4 + c, n_x) || !INV_IN_BOUNDS(status, r * ldo4 + c, n_out)) continue;
     const float4 v = x[r * ld4 + c];
     __half h[4], l[4];
     split_hi_lo(v.x, h[0], l[0]);
@@ -68,9 +70,10 @@ __global__ void heal_split_vec_kernel(const float4* __restrict__ x, int64_t rows
 
 // Column exponent: max_k |W[k][n]| 2^e in [2^14, 2^15); one thread per column,
 // consecutive threads read consecutive columns of a row (coalesced).
-__global__ void col_exp_kernel(const float* __restrict__ W, int K, int N, int8_t* __restrict__ e_out) {
+__global__ void col_exp_kernel(const float* __restrict__ W, int K, int N, int8_t* __restrict__ e_out, int* status) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= N) return;
+  if (!INV_SPAN_IN_BOUNDS(status, n, (int64_t)(K - 1) * N + n, (int64_t)K * N) || !INV_IN_BOUNDS(status, n, N)) return;
   float m = 0.0f;
   for (int k = 0; k < K; ++k) m = fmaxf(m, fabsf(W[(int64_t)k * N + n]));
   int e = 0;
@@ -85,23 +88,29 @@ __global__ void col_exp_kernel(const float* __restrict__ W, int K, int N, int8_t
 
 // Packed image [N/128][2][128][K]; a block transposes a 64(k) x 64(n) tile.
 __global__ void pack_kernel(const float* __restrict__ W, int K, int N, const int8_t* __restrict__ e,
-                            __half* __restrict__ P) {
+                            __half* __restrict__ P, int* status) {
   constexpr int PW = INV_GEMM_BN;    // panel width
   __shared__ float tile[64][65];
   const int n0 = blockIdx.x * 64;    // 64 columns, inside one panel
   const int k0 = blockIdx.y * 64;
   const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 256 threads: 64 x 4
-  for (int kk = ty; kk < 64; kk += 4) tile[kk][tx] = W[(int64_t)(k0 + kk) * N + n0 + tx];
+  [[maybe_unused]] const int64_t n_w = (int64_t)K * N, n_p = 2 * (int64_t)K * N;
+  for (int kk = ty; kk < 64; kk += 4) {
+    const int64_t iw = (int64_t)(k0 + kk) * N + n0 + tx;
+    tile[kk][tx] = INV_IN_BOUNDS(status, iw, n_w) ? W[iw] : 0.0f;
+  }
   __syncthreads();
   for (int r = ty; r < 64; r += 4) {
     const int n = n0 + r;
     const int j = n / PW, rr = n % PW;
+    if (!INV_IN_BOUNDS(status, n, N)) continue;
     const float s = inv::pow2f(e[n]);
     const float v = __fmul_rn(tile[tx][r], s);  // exact power-of-two scaling
     __half h, l;
     split_hi_lo(v, h, l);
-    P[(((int64_t)j * 2 + 0) * PW + rr) * K + k0 + tx] = h;
-    P[(((int64_t)j * 2 + 1) * PW + rr) * K + k0 + tx] = l;
+    const int64_t ih = (((int64_t)j * 2 + 0) * PW + rr) * K + k0 + tx, il = ih + (int64_t)PW * K;
+    if (INV_IN_BOUNDS(status, ih, n_p)) P[ih] = h;
+    if (INV_IN_BOUNDS(status, il, n_p)) P[il] = l;
   }
 }
 
@@ -119,6 +128,8 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* __re
   __shared__ float warp_sum[kNormThreads / 32];
   __shared__ float r_sh;
   const int64_t row = blockIdx.x;
+  // x and the outputs are [rows = gridDim.x][hidden]; the row is accessed whole
+  if (!INV_SPAN_IN_BOUNDS(status, row * hidden, row * hidden + hidden - 1, (int64_t)gridDim.x * hidden)) return;
   const float4* xr = reinterpret_cast<const float4*>(x + row * hidden);
   const int n4 = hidden / 4;
   float s = 0.0f;
@@ -183,6 +194,8 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_reg_kernel(const float* 
   __shared__ float warp_sum[kNormThreads / 32];
   __shared__ float r_sh;
   const int64_t row = blockIdx.x;
+  // x and the outputs are [rows = gridDim.x][hidden]; the row is accessed whole
+  if (!INV_SPAN_IN_BOUNDS(status, row * hidden, row * hidden + hidden - 1, (int64_t)gridDim.x * hidden)) return;
   const float4* xr = reinterpret_cast<const float4*>(x + row * hidden);
   const int n4 = hidden / 4;
   const float4* g4 = reinterpret_cast<const float4*>(gamma);
@@ -284,8 +297,13 @@ __global__ void kv_quant_kernel(const float* __restrict__ x, int T, int64_t ld_x
     if (lane == 0) record_status(status, INV_ERR_INVALID_ARG);
     return;
   }
-  const float4 v = reinterpret_cast<const float4*>(x + (int64_t)t * ld_x + (int64_t)h * 128)[lane];
+  const int64_t ix = (int64_t)t * ld_x + (int64_t)h * 128;
   const int64_t rowi = ((int64_t)sl * H + h) * c.max_len + p;
+  [[maybe_unused]] const int64_t n_rows = (int64_t)c.n_slots * H * c.max_len;  // cache rows
+  if (!INV_SPAN_IN_BOUNDS(status, ix, ix + 127, (int64_t)(T - 1) * ld_x + (int64_t)H * 128) ||
+      !INV_IN_BOUNDS(status, rowi, n_rows))
+    return;
+  const float4 v = reinterpret_cast<const float4*>(x + ix)[lane];
   int16_t* codes = (which == 0 ? c.k : c.v) + rowi * 128;
   float* scale = (which == 0 ? c.k_scale : c.v_scale) + rowi;
   quant_store_row(v, codes, scale, lane);
@@ -328,7 +346,8 @@ __global__ void rope_quant_kernel(const float* __restrict__ qkv, int T, int Hq, 
                                   int64_t n_a, int* status) {
   {
     const int64_t t0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x, stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = t0; i < n_a; i += stride) zero_a[i] = 0;
+    for (int64_t i = t0; i < n_a; i += stride)
+      if (INV_IN_BOUNDS(status, i, n_a)) zero_a[i] = 0;
   }
   const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -338,20 +357,27 @@ __global__ void rope_quant_kernel(const float* __restrict__ qkv, int T, int Hq, 
   const int t = (int)(warp / nh), hi = (int)(warp - (int64_t)t * nh);
   const int sl = slot[t], p = pos[t];
   const bool ok = sl >= 0 && sl < c.n_slots && p >= 0 && p < c.max_len && p < max_pos;
-  if (hi == 0 && lane == 0) len_out[t] = ok ? p + 1 : 0;
+  if (hi == 0 && lane == 0 && INV_IN_BOUNDS(status, t, T)) len_out[t] = ok ? p + 1 : 0;
   if (!ok) {
     if (lane == 0 && hi == 0) record_status(status, INV_ERR_INVALID_ARG);
     return;
   }
-  float4 v = reinterpret_cast<const float4*>(qkv + (int64_t)t * nh * 128 + (int64_t)hi * 128)[lane];
+  const int64_t iq = (int64_t)t * nh * 128 + (int64_t)hi * 128;
+  if (!INV_SPAN_IN_BOUNDS(status, iq, iq + 127, (int64_t)T * nh * 128) ||
+      !INV_SPAN_IN_BOUNDS(status, (int64_t)p * 64, (int64_t)p * 64 + 63, (int64_t)max_pos * 64))
+    return;
+  float4 v = reinterpret_cast<const float4*>(qkv + iq)[lane];
   if (hi < Hq + Hkv) v = rope_row(v, rope_cos + (int64_t)p * 64, rope_sin + (int64_t)p * 64, lane);
   if (hi < Hq) {
-    reinterpret_cast<float4*>(q_out + ((int64_t)t * Hq + hi) * 128)[lane] = v;
+    const int64_t io = ((int64_t)t * Hq + hi) * 128;
+    if (INV_SPAN_IN_BOUNDS(status, io, io + 127, (int64_t)T * Hq * 128))
+      reinterpret_cast<float4*>(q_out + io)[lane] = v;
     return;
   }
   const bool is_k = hi < Hq + Hkv;
   const int h = is_k ? hi - Hq : hi - Hq - Hkv;
   const int64_t rowi = ((int64_t)sl * Hkv + h) * c.max_len + p;
+  if (!INV_IN_BOUNDS(status, rowi, (int64_t)c.n_slots * Hkv * c.max_len)) return;
   quant_store_row(v, (is_k ? c.k : c.v) + rowi * 128, (is_k ? c.k_scale : c.v_scale) + rowi, lane);
 }
 
@@ -361,18 +387,24 @@ __global__ void embed_kernel(const float* __restrict__ table, int vocab, int hid
   const int id = ids[b];
   const bool ok = id >= 0 && id < vocab;
   if (!ok && threadIdx.x == 0) record_status(status, INV_ERR_INVALID_ARG);
-  for (int i = threadIdx.x; i < hidden; i += blockDim.x)
-    x[(int64_t)b * hidden + i] = ok ? table[(int64_t)id * hidden + i] : 0.0f;
+  for (int i = threadIdx.x; i < hidden; i += blockDim.x) {
+    const int64_t ix = (int64_t)b * hidden + i, it = (int64_t)id * hidden + i;
+    if (!INV_IN_BOUNDS(status, ix, (int64_t)B * hidden) || (ok && !INV_IN_BOUNDS(status, it, (int64_t)vocab * hidden)))
+      continue;
+    x[ix] = ok ? table[it] : 0.0f;
+  }
 }
 
 // Greedy argmax per row: lowest index among the maxima (NaN ignored).
-__global__ void argmax_kernel(const float* __restrict__ logits, int n, int64_t ld, int32_t* __restrict__ ids) {
+__global__ void argmax_kernel(const float* __restrict__ logits, int n, int64_t ld, int32_t* __restrict__ ids,
+                              int* status) {
   __shared__ float bv[32];
   __shared__ int bi[32];
-  const int64_t b = blockIdx.x;
+  const int64_t b = blockIdx.x;  // logits [B = gridDim.x] rows of ld, the last one n long
   float best = -INFINITY;
   int besti = 0x7fffffff;
   for (int j = threadIdx.x; j < n; j += blockDim.x) {
+    if (!INV_IN_BOUNDS(status, b * ld + j, ((int64_t)gridDim.x - 1) * ld + n)) continue;
     const float v = logits[b * ld + j];
     if (v > best || (v == best && j < besti)) { best = v; besti = j; }
   }
@@ -386,14 +418,15 @@ __global__ void argmax_kernel(const float* __restrict__ logits, int n, int64_t l
   if (threadIdx.x == 0) {
     for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
       if (bv[w] > best || (bv[w] == best && bi[w] < besti)) { best = bv[w]; besti = bi[w]; }
-    ids[b] = besti == 0x7fffffff ? 0 : besti;
+    if (INV_IN_BOUNDS(status, b, gridDim.x)) ids[b] = besti == 0x7fffffff ? 0 : besti;
   }
 }
 
 // cos/sin(p * base^(-2i/128)) in double precision, rounded once to fp32.
-__global__ void rope_table_kernel(int max_pos, double base, float* __restrict__ cs, float* __restrict__ sn) {
+__global__ void rope_table_kernel(int max_pos, double base, float* __restrict__ cs, float* __restrict__ sn,
+                                  int* status) {
   const int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (idx >= (int64_t)max_pos * 64) return;
+  if (idx >= (int64_t)max_pos * 64 || !INV_IN_BOUNDS(status, idx, (int64_t)max_pos * 64)) return;
   const int p = (int)(idx / 64), i = (int)(idx % 64);
   const double theta = pow(base, -2.0 * i / 128.0);
   double sv, cv;
@@ -487,9 +520,10 @@ int heal_pack_weight(const float* W, int K, int N, uint16_t* packed, size_t pack
   if (K % 64 != 0 || N % INV_GEMM_BN != 0) return INV_ERR_UNSUPPORTED_SHAPE;
   if (packed_bytes < heal_packed_weight_bytes(K, N)) return INV_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  col_exp_kernel<<<(N + 255) / 256, 256, 0, s>>>(W, K, N, col_exp);
+  col_exp_kernel<<<(N + 255) / 256, 256, 0, s>>>(W, K, N, col_exp, inv::status_ptr());
   INV_CHECK_LAUNCH();
-  pack_kernel<<<dim3(N / 64, K / 64), 256, 0, s>>>(W, K, N, col_exp, reinterpret_cast<__half*>(packed));
+  pack_kernel<<<dim3(N / 64, K / 64), 256, 0, s>>>(W, K, N, col_exp, reinterpret_cast<__half*>(packed),
+                                                   inv::status_ptr());
   INV_CHECK_LAUNCH();
   return INV_OK;
 }
@@ -526,8 +560,8 @@ int kv_quant_int16(const float* x, int T, int64_t ld_x, const int32_t* slot, con
 int rope_tables(int max_pos, double base, float* cos_out, float* sin_out, inv_stream stream) {
   if (max_pos <= 0 || !(base > 0.0) || !cos_out || !sin_out) return INV_ERR_INVALID_ARG;
   const int64_t n = (int64_t)max_pos * 64;
-  rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(max_pos, base, cos_out,
-                                                                                                 sin_out);
+  rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      max_pos, base, cos_out, sin_out, inv::status_ptr());
   INV_CHECK_LAUNCH();
   return INV_OK;
 }
@@ -545,7 +579,7 @@ int argmax_rows(const float* logits, int B, int n, int64_t ld, int32_t* ids, inv
   if (B < 0 || n <= 0 || ld < n) return INV_ERR_INVALID_ARG;
   if (B == 0) return INV_OK;
   if (!logits || !ids) return INV_ERR_INVALID_ARG;
-  argmax_kernel<<<B, 1024, 0, static_cast<cudaStream_t>(stream)>>>(logits, n, ld, ids);
+  argmax_kernel<<<B, 1024, 0, static_cast<cudaStream_t>(stream)>>>(logits, n, ld, ids, inv::status_ptr());
   INV_CHECK_LAUNCH();
   return INV_OK;
 }

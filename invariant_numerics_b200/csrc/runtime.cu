@@ -114,6 +114,15 @@ __global__ void selftest_wait_kernel(int* status, long long limit_ns) {
   __syncthreads();
 }
 
+// Stores i to buf[i] for i < n_written under the index check with extent
+// n_declared (launched only by the checking build).
+__global__ void selftest_bounds_kernel(float* buf, int n_declared, int n_written, int* status) {
+#ifdef INV_DEBUG_BOUNDS
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_written; i += gridDim.x * blockDim.x)
+    if (INV_IN_BOUNDS(status, i, n_declared)) buf[i] = (float)i;
+#endif
+}
+
 }  // namespace
 
 extern "C" {
@@ -127,6 +136,7 @@ const char* inv_status_string(int status) {
     case INV_ERR_CUDA: return "INV_ERR_CUDA";
     case INV_ERR_RANGE: return "INV_ERR_RANGE";
     case INV_ERR_TIMEOUT: return "INV_ERR_TIMEOUT";
+    case INV_ERR_BOUNDS: return "INV_ERR_BOUNDS";
     default: return "INV_ERR_UNKNOWN";
   }
 }
@@ -166,6 +176,26 @@ int inv_selftest_wait_timeout(long long wait_ns, inv_stream stream) {
   int* st = inv::status_ptr();
   if (st == nullptr) return INV_ERR_CUDA;
   selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(st, wait_ns);
+  INV_CHECK_LAUNCH();
+  return INV_OK;
+}
+
+int inv_debug_bounds_enabled(void) {
+#ifdef INV_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+int inv_selftest_bounds(float* buf, int n_declared, int n_written, inv_stream stream) {
+  if (buf == nullptr || n_declared < 0 || n_written < n_declared) return INV_ERR_INVALID_ARG;
+  if (!inv_debug_bounds_enabled()) return INV_ERR_UNSUPPORTED_SHAPE;
+  if (n_written == 0) return INV_OK;
+  int* st = inv::status_ptr();
+  if (st == nullptr) return INV_ERR_CUDA;
+  selftest_bounds_kernel<<<(n_written + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(buf, n_declared,
+                                                                                                 n_written, st);
   INV_CHECK_LAUNCH();
   return INV_OK;
 }

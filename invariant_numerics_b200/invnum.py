@@ -16,13 +16,16 @@ from dataclasses import dataclass, field
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libinvnum.so")
+# INVNUM_LIBRARY may name another build of the same library (the
+# index-checking libinvnum_debug.so); by default the package's libinvnum.so.
+_LIB_PATH = os.environ.get("INVNUM_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                                                              "libinvnum.so")
 if not os.path.exists(_LIB_PATH):
     raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m invariant_numerics_b200.build`")
 lib = C.CDLL(_LIB_PATH)
 
 INV_OK, INV_ERR_INVALID_ARG, INV_ERR_UNSUPPORTED_SHAPE, INV_ERR_WORKSPACE, INV_ERR_CUDA, INV_ERR_RANGE, \
-    INV_ERR_TIMEOUT = range(7)
+    INV_ERR_TIMEOUT, INV_ERR_BOUNDS = range(8)
 KV_SPLIT = 256
 HEAD_DIM = 128
 
@@ -57,6 +60,8 @@ _SIGS = {
     "inv_get_device_status": (_i, [C.POINTER(_i), _p]),
     "inv_set_wait_limit_ns": (_i, [C.c_longlong]),
     "inv_selftest_wait_timeout": (_i, [C.c_longlong, _p]),
+    "inv_debug_bounds_enabled": (_i, []),
+    "inv_selftest_bounds": (_i, [_p, _i, _i, _p]),
     "inv_selftest_gemm_wait_timeout": (_i, [_p, _sz, C.c_longlong, _p]),
     "inv_trace_events": (_i, [C.POINTER(C.c_void_p), _i]),
     "heal_split": (_i, [_p, _i64, _i64, _i64, _p, _p, _i64, _p]),
@@ -147,6 +152,17 @@ def inv_selftest_gemm_wait_timeout(wait_ns: int, workspace=None, stream=None) ->
     ws = torch.empty(SELFTEST_GEMM_WS_BYTES, dtype=torch.uint8, device="cuda") if workspace is None else workspace
     _check("inv_selftest_gemm_wait_timeout",
            lib.inv_selftest_gemm_wait_timeout(_ptr(ws), ws.numel(), int(wait_ns), _stream(stream)))
+
+
+def inv_debug_bounds_enabled() -> bool:
+    return bool(lib.inv_debug_bounds_enabled())
+
+
+def inv_selftest_bounds(buf, n_declared: int, n_written: int, stream=None) -> None:
+    _need(buf, torch.float32, "buf")
+    if buf.numel() < n_declared:
+        raise ValueError("buf must hold n_declared floats")
+    _check("inv_selftest_bounds", lib.inv_selftest_bounds(_ptr(buf), int(n_declared), int(n_written), _stream(stream)))
 
 
 DECODE_LAYER_KERNELS = 9

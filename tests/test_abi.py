@@ -64,3 +64,27 @@ def test_binding_module_exposes_the_same_names():
               "rmsnorm_bi", "decode_layer", "rope_tables", "embed_gather", "argmax_rows",
               "inv_get_device_status", "inv_set_wait_limit_ns", "inv_selftest_wait_timeout"):
         assert callable(getattr(inv, n)), n
+
+
+@pytest.fixture(scope="module")
+def debug_lib():
+    from invariant_numerics_b200 import build
+    path = build.build(debug_bounds=True)
+    return ctypes.CDLL(path), path
+
+
+def test_index_checking_build_exports_the_same_symbols(lib, debug_lib):
+    L, path = lib
+    D, dpath = debug_lib
+    nm = lambda p: {ln.split()[-1] for ln in subprocess.run(["nm", "-D", "--defined-only", p], capture_output=True,
+                                                             text=True).stdout.splitlines() if " T " in ln}
+    assert set(declared_functions()) <= nm(dpath)
+    assert {s for s in nm(dpath) if not s.startswith("_") and not s.startswith("cu")} <= set(declared_functions())
+    assert L.inv_debug_bounds_enabled() == 0 and D.inv_debug_bounds_enabled() == 1
+    L.inv_status_string.restype = ctypes.c_char_p
+    assert L.inv_status_string(7) == b"INV_ERR_BOUNDS"
+    # the normal build refuses the self-test (its stores would be unchecked) without touching the GPU
+    buf = ctypes.c_void_p(16)
+    assert L.inv_selftest_bounds(buf, 4, 8, None) == 2  # INV_ERR_UNSUPPORTED_SHAPE
+    assert L.inv_selftest_bounds(buf, 8, 4, None) == 1  # n_written < n_declared
+    assert D.inv_selftest_bounds(None, 4, 8, None) == 1
