@@ -52,7 +52,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # profiles/dram_traffic.txt together with the SHA-256 of the kernel's source
 # file at capture time: a record whose source has changed since is not used.
 TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-KERNEL_SOURCES = {"comp_gemm_kernel": "comp_gemm.cu", "attn_split_kernel": "attention.cu"}
+KERNEL_SOURCES = {"comp_gemm_kernel": "comp_gemm.cu", "qkv_attn_kernel": "comp_gemm.cu",
+                  "attn_split_kernel": "attention.cu"}
 
 
 def captured_traffic(kernel: str, workload: str):
@@ -410,7 +411,9 @@ def layer_bytes(B, L):
     """Algorithmic HBM bytes of one decode-layer step and of its kernels."""
     Nqkv = (HQ + 2 * HKV) * D
     gemm = {  # packed weights (4 B / weight) + A hi/lo (4 B / element) + y fp32 (+ residual fp32)
-        "gemm_qkv": 4 * H * Nqkv + 4 * B * H + 4 * B * Nqkv,
+        # QKV: its epilogue writes rotated q (fp32), the new K/V rows of the
+        # cache (INT16 codes + fp32 scale) and reads the rows' rotary tables
+        "gemm_qkv_rope_quant": 4 * H * Nqkv + 4 * B * H + 4 * B * HQ * D + B * 2 * HKV * (2 * D + 4) + B * 2 * 64 * 4,
         "gemm_o": 4 * HQ * D * H + 4 * B * HQ * D + 8 * B * H,
         "gemm_gate_up_swiglu": 4 * H * 2 * F + 4 * B * H + 4 * B * F,
         "gemm_down": 4 * F * H + 4 * B * F + 8 * B * H,
@@ -609,7 +612,12 @@ def run_ours(args, rank, world, local):
                 "algorithmic_bytes_per_launch": round(byts_per_step / launches),
                 "us_per_launch": round(us / launches, 2), "share_of_traced_step": round(us / traced_us, 4),
                 "peak_source": f"{peak_kind} hbm_gbs"}
-    lines = sorted([roofline_of("comp_gemm_kernel", list(gemm_b), sum(gemm_b.values())),
+    # kernel functions: comp_gemm_kernel (o, gate/up + SwiGLU, down), the QKV
+    # GEMM with the fused rotary/quantise epilogue (qkv_attn_kernel), the
+    # attention split kernel
+    plain = [n for n in gemm_b if n != "gemm_qkv_rope_quant"]
+    lines = sorted([roofline_of("comp_gemm_kernel", plain, sum(gemm_b[n] for n in plain)),
+                    roofline_of("qkv_attn_kernel", ["gemm_qkv_rope_quant"], gemm_b["gemm_qkv_rope_quant"]),
                     roofline_of("attn_split_kernel", ["attn_split"], attn_b)],
                    key=lambda r: -r["share_of_traced_step"])
     step_bytes = sum(gemm_b.values()) + attn_b
@@ -631,6 +639,7 @@ def run_ours(args, rank, world, local):
                    "l2": "inputs larger than L2 (708.8 MB packed weights + 1.09 GB INT16 KV per step)"},
         "roofline": lines[0],
         "roofline_second": lines[1],
+        "roofline_others": lines[2:],
         "step_roofline": {"bytes": step_bytes, "hbm_bound_ms": round(step_bytes / (hbm * 1e9) * 1e3, 4),
                           "frac": round(step_bytes / (hbm * 1e9) * 1e3 / ms, 4)},
         "kernels": kernels,

@@ -141,12 +141,13 @@ INV_API int inv_selftest_bounds(float* buf, int n_declared, int n_written, inv_s
  * Kernel tracing for decode_layer (profiling aid; off by default).  With
  * events != NULL and n_events >= 2 * INV_DECODE_LAYER_KERNELS, every later
  * decode_layer call records events[2i] before and events[2i+1] after its i-th
- * kernel launch, on the call's stream (i: 0 rmsnorm, 1 qkv GEMM, 2 rotary +
- * quantise, 3 attention splits, 4 attention combine, 5 output GEMM, 6 rmsnorm,
- * 7 gate/up GEMM with fused SwiGLU, 8 down GEMM).  events are cudaEvent_t
- * handles the caller created and keeps alive.  NULL / 0 switches tracing off.  Host-global.
+ * kernel launch, on the call's stream (i: 0 rmsnorm, 1 qkv GEMM with the
+ * rotary embedding and the KV quantiser in its epilogue, 2 attention splits,
+ * 3 attention combine, 4 output GEMM, 5 rmsnorm, 6 gate/up GEMM with fused
+ * SwiGLU, 7 down GEMM).  events are cudaEvent_t handles the caller created
+ * and keeps alive.  NULL / 0 switches tracing off.  Host-global.
  */
-#define INV_DECODE_LAYER_KERNELS 9
+#define INV_DECODE_LAYER_KERNELS 8
 INV_API int inv_trace_events(void** events, int n_events);
 
 /* ------------------------------------------------------------------------
@@ -344,6 +345,9 @@ INV_API int rmsnorm_bi(const float* x, const float* gamma, int64_t rows, int hid
  *   qkv = comp_gemm(h, W_qkv)                         (N = (Hq + 2 Hkv) 128)
  *   q, k <- rotary embedding (rotate-half, pairs (i, i+64), tables below)
  *   k, v -> kv_quant_int16 into (slot[b], pos[b])     (all rows before any attention)
+ *        (these three run as one kernel: the GEMM's epilogue rotates and
+ *        quantises each 128-wide head tile in fp32, the same operations in
+ *        the same order as the separate steps)
  *   o  = attn_decode_fixedsplit(q, len = pos + 1)    -> hi/lo
  *   x1 = x + comp_gemm(o, W_o)
  *   h2 = rmsnorm_bi(x1, g_mlp)                       -> hi/lo
@@ -360,8 +364,8 @@ INV_API int rmsnorm_bi(const float* x, const float* gamma, int64_t rows, int hid
  *                 cache->max_len when max_len_bound <= 0 (the size function
  *                 returns 0 for L <= 0).  Calls that overlap on the GPU need
  *                 separate workspaces.
- * Stream work: the layer's kernels only, all on `stream` (the rotary/quantise
- * kernel also clears the workspace's gate/up tile counters).  The W_down GEMM
+ * Stream work: the layer's kernels only, all on `stream` (the QKV GEMM also
+ * clears the workspace's gate/up tile counters).  The W_down GEMM
  * is launched as a
  * programmatic dependent of the gate/up GEMM and starts during its last
  * partial wave, loading each K block of a once the gate/up tile that stores it

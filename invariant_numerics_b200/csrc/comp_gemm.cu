@@ -66,6 +66,14 @@ struct __align__(1024) GemmSmem {
   int abort;
 };
 constexpr size_t kSmemBytes = sizeof(GemmSmem) + 1024;
+// The fused attention-input epilogue also needs, after GemmSmem, the per-row
+// max |x| of each half of a head: [2][BM] floats.  (Measured: 198.7 KB of
+// dynamic shared memory plus the 1 KB each CTA reserves fills the 196 KB
+// shared-memory configuration exactly; 1 KB more still fits it, while 2 KB
+// more moved every GEMM to the next configuration and made it 1-2 us slower.)
+constexpr size_t kRowMaxBytes = 2 * BM * sizeof(float);
+template <bool kAttnIn>
+constexpr size_t smem_bytes() { return kSmemBytes + (kAttnIn ? kRowMaxBytes : 0); }
 
 // Consumer side of a producer/consumer GEMM pair: ready_row[kb] counts the
 // epilogue warps of the producing grid that have stored (and released) the
@@ -107,13 +115,30 @@ __device__ bool wait_published(const int* ready_row, int kb, int nkb, int* upto,
   }
 }
 
-template <int BN>
-__global__ void __launch_bounds__(THREADS, 1)
-    comp_gemm_kernel(const __grid_constant__ CUtensorMap tm_ahi, const __grid_constant__ CUtensorMap tm_alo,
-                     const __grid_constant__ CUtensorMap tm_w, const int8_t* __restrict__ col_exp, float* y,
-                     int64_t ld_y, const float* residual, int64_t ld_r, __half* gate_hi, __half* gate_lo,
-                     int64_t ld_g, int M, int N, int K, int box_rows, int a_stride, int n_stages, int* ready_out,
-                     const int* ready_in, int* status, long long wait_ns) {
+// AND of v over the 64 threads (two warps) at named barrier `id`.
+__device__ __forceinline__ bool pair_all(bool v, int id) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, 64, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u), "r"(id)
+      : "memory");
+  return r != 0;
+}
+
+// The kernel body; comp_gemm_kernel and qkv_attn_kernel (the fused
+// attention-input epilogue, kAttnIn) are its two entry points, so that the
+// plain GEMM's parameter list carries nothing it does not use.
+template <int BN, bool kAttnIn>
+__device__ __forceinline__ void gemm_body(const CUtensorMap& tm_ahi, const CUtensorMap& tm_alo,
+                                          const CUtensorMap& tm_w, const int8_t* __restrict__ col_exp, float* y,
+                                          int64_t ld_y, const float* residual, int64_t ld_r, __half* gate_hi,
+                                          __half* gate_lo, int64_t ld_g, int M, int N, int K, int box_rows,
+                                          int a_stride, int n_stages, int* ready_out, const int* ready_in,
+                                          int* status, long long wait_ns, const inv::AttnInputs& ai) {
   using T = Tile<BN>;
   constexpr int W_BYTES = T::W_BYTES, ACC_COLS = T::ACC_COLS, TMEM_COLS = T::TMEM_COLS, EPI_COLS = T::EPI_COLS;
   extern __shared__ uint8_t smem_raw[];
@@ -228,123 +253,287 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue --
-    const int quarter = warp & 3;          // TMEM lanes 32*quarter .. +31
-    const int half = (warp - 2) >> 2;      // output columns EPI_COLS*half .. +EPI_COLS-1
-    uint32_t g = 0;
-    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-      const int nt = tile / tiles_m, mt = tile - nt * tiles_m;
-      float acc_h[EPI_COLS], acc_x[EPI_COLS];
+    // Warp w drains TMEM lanes 32*(w%4).. (its 32 rows) and half of the tile's
+    // columns: half = (w-2)/4 takes [half EPI_COLS, +EPI_COLS); with the fused
+    // attention inputs (the second loop below) instead [half BN/4, +BN/4) and
+    // [BN/2 + half BN/4, +BN/4), so that a thread holds columns j and j + BN/2
+    // of its row (the rotate-half partners of a 128-wide head); there local
+    // column c < EPI_COLS maps to tile column tcol(c).
+    if constexpr (!kAttnIn) {
+      const int quarter = warp & 3;          // TMEM lanes 32*quarter .. +31
+      const int half = (warp - 2) >> 2;      // output columns EPI_COLS*half .. +EPI_COLS-1
+      uint32_t g = 0;
+      for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        const int nt = tile / tiles_m, mt = tile - nt * tiles_m;
+        float acc_h[EPI_COLS], acc_x[EPI_COLS];
 #pragma unroll
-      for (int i = 0; i < EPI_COLS; ++i) acc_h[i] = acc_x[i] = 0.0f;
-      for (int grp = 0; grp < ngroups; ++grp, ++g) {
-        const uint32_t buf = g & 1u, tph = (g >> 1) & 1u;
-        int okw = 1;
-        if (lane == 0) okw = inv::mbar_wait(&sm.tfull[buf], tph, wait_ns, abort_flag, status) ? 1 : 0;
-        okw = __shfl_sync(0xffffffffu, okw, 0);  // keep the warp converged for tcgen05.ld
-        if (!okw) goto epi_done;
-        inv::tc_fence_after();
-        const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * ACC_COLS + half * EPI_COLS;
+        for (int i = 0; i < EPI_COLS; ++i) acc_h[i] = acc_x[i] = 0.0f;
+        for (int grp = 0; grp < ngroups; ++grp, ++g) {
+          const uint32_t buf = g & 1u, tph = (g >> 1) & 1u;
+          int okw = 1;
+          if (lane == 0) okw = inv::mbar_wait(&sm.tfull[buf], tph, wait_ns, abort_flag, status) ? 1 : 0;
+          okw = __shfl_sync(0xffffffffu, okw, 0);  // keep the warp converged for tcgen05.ld
+          if (!okw) goto epi_done;
+          inv::tc_fence_after();
+          const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * ACC_COLS + half * EPI_COLS;
 #pragma unroll
-        for (int c = 0; c < EPI_COLS; c += 16) {
-          uint32_t rh[16], rx[16];
-          inv::tmem_ld_32x16(ta + c, rh);
-          inv::tmem_ld_32x16(ta + BN + c, rx);
-          inv::tmem_wait_ld();
+          for (int c = 0; c < EPI_COLS; c += 16) {
+            uint32_t rh[16], rx[16];
+            inv::tmem_ld_32x16(ta + c, rh);
+            inv::tmem_ld_32x16(ta + BN + c, rx);
+            inv::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            acc_h[c + i] = __fadd_rn(acc_h[c + i], __uint_as_float(rh[i]));
-            acc_x[c + i] = __fadd_rn(acc_x[c + i], __uint_as_float(rx[i]));
+            for (int i = 0; i < 16; ++i) {
+              acc_h[c + i] = __fadd_rn(acc_h[c + i], __uint_as_float(rh[i]));
+              acc_x[c + i] = __fadd_rn(acc_x[c + i], __uint_as_float(rx[i]));
+            }
           }
+          inv::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) inv::mbar_arrive(&sm.tempty[buf]);
         }
-        inv::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) inv::mbar_arrive(&sm.tempty[buf]);
-      }
-      {
-        const int row = mt * BM + quarter * 32 + lane;
-        const int col0 = nt * BN + half * EPI_COLS;
-        if (row < M && gate_hi != nullptr) {
-          // Fused SwiGLU: each 32 packed columns are 16 gate columns then the
-          // 16 matching up columns of outputs f0 .. f0+15, f0 = column / 2
-          // (a panel of BN >= 64 columns; the host never asks for less).
+        {
+          const int row = mt * BM + quarter * 32 + lane;
+          const int col0 = nt * BN + half * EPI_COLS;
+          if (row < M && gate_hi != nullptr) {
+            // Fused SwiGLU: each 32 packed columns are 16 gate columns then the
+            // 16 matching up columns of outputs f0 .. f0+15, f0 = column / 2
+            // (a panel of BN >= 64 columns; the host never asks for less).
 #pragma unroll
-          for (int c = 0; c < (EPI_COLS % 32 == 0 ? EPI_COLS : 0); c += 32) {
-            const int f0 = (col0 + c) / 2;
-            // index checks: 32 column exponents, 16 outputs of gate_hi/lo [M][ld_g] (N / 2 used)
-            if (!INV_SPAN_IN_BOUNDS(status, col0 + c, col0 + c + 31, N) ||
-                !INV_SPAN_IN_BOUNDS(status, (int64_t)row * ld_g + f0, (int64_t)row * ld_g + f0 + 15,
-                                    (int64_t)(M - 1) * ld_g + N / 2))
-              continue;
-            float v[32];
+            for (int c = 0; c < (EPI_COLS % 32 == 0 ? EPI_COLS : 0); c += 32) {
+              const int f0 = (col0 + c) / 2;
+              // index checks: 32 column exponents, 16 outputs of gate_hi/lo [M][ld_g] (N / 2 used)
+              if (!INV_SPAN_IN_BOUNDS(status, col0 + c, col0 + c + 31, N) ||
+                  !INV_SPAN_IN_BOUNDS(status, (int64_t)row * ld_g + f0, (int64_t)row * ld_g + f0 + 15,
+                                      (int64_t)(M - 1) * ld_g + N / 2))
+                continue;
+              float v[32];
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              const char4 e4 = *reinterpret_cast<const char4*>(col_exp + col0 + c + i);
+              for (int i = 0; i < 32; i += 4) {
+                const char4 e4 = *reinterpret_cast<const char4*>(col_exp + col0 + c + i);
+                const int ev[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const float t = __fadd_rn(acc_h[c + i + j], __fmul_rn(acc_x[c + i + j], 0x1p-11f));
+                  v[i + j] = __fmul_rn(t, inv::pow2f(-ev[j]));
+                }
+              }
+              uint32_t hw[8], lw[8];
+              bool bad = false;
+#pragma unroll
+              for (int i = 0; i < 16; i += 2) {
+                __half h0, l0, h1, l1;
+                const float a0 = __fmul_rn(__fdiv_rn(v[i], __fadd_rn(1.0f, expf(-v[i]))), v[16 + i]);
+                const float a1 = __fmul_rn(__fdiv_rn(v[i + 1], __fadd_rn(1.0f, expf(-v[i + 1]))), v[17 + i]);
+                bad |= inv::f16_overflow(a0) | inv::f16_overflow(a1);
+                inv::split_hi_lo(a0, h0, l0);
+                inv::split_hi_lo(a1, h1, l1);
+                hw[i / 2] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
+                lw[i / 2] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
+              }
+              if (bad) inv::record_status(status, INV_ERR_RANGE);
+              uint4* gh = reinterpret_cast<uint4*>(gate_hi + (int64_t)row * ld_g + f0);
+              uint4* gl = reinterpret_cast<uint4*>(gate_lo + (int64_t)row * ld_g + f0);
+              gh[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              gh[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+              gl[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+              gl[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+            }
+          } else if (row < M &&
+                     INV_SPAN_IN_BOUNDS(status, col0, col0 + EPI_COLS - 1, N) &&
+                     INV_SPAN_IN_BOUNDS(status, (int64_t)row * ld_y + col0, (int64_t)row * ld_y + col0 + EPI_COLS - 1,
+                                        (int64_t)(M - 1) * ld_y + N) &&
+                     (residual == nullptr ||
+                      INV_SPAN_IN_BOUNDS(status, (int64_t)row * ld_r + col0, (int64_t)row * ld_r + col0 + EPI_COLS - 1,
+                                         (int64_t)(M - 1) * ld_r + N))) {
+            // (index checks above: column exponents, y [M][ld_y] and residual [M][ld_r], N columns used)
+            float* yr = y + (int64_t)row * ld_y + col0;
+            const float* rr = residual ? residual + (int64_t)row * ld_r + col0 : nullptr;
+#pragma unroll
+            for (int i = 0; i < EPI_COLS; i += 4) {
+              const char4 e4 = *reinterpret_cast<const char4*>(col_exp + col0 + i);
               const int ev[4] = {e4.x, e4.y, e4.z, e4.w};
+              float o[4];
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const float t = __fadd_rn(acc_h[c + i + j], __fmul_rn(acc_x[c + i + j], 0x1p-11f));
-                v[i + j] = __fmul_rn(t, inv::pow2f(-ev[j]));
+                const float t = __fadd_rn(acc_h[i + j], __fmul_rn(acc_x[i + j], 0x1p-11f));
+                o[j] = __fmul_rn(t, inv::pow2f(-ev[j]));
               }
+              if (rr) {
+                const float4 r4 = *reinterpret_cast<const float4*>(rr + i);
+                o[0] = __fadd_rn(o[0], r4.x);
+                o[1] = __fadd_rn(o[1], r4.y);
+                o[2] = __fadd_rn(o[2], r4.z);
+                o[3] = __fadd_rn(o[3], r4.w);
+              }
+              *reinterpret_cast<float4*>(yr + i) = make_float4(o[0], o[1], o[2], o[3]);
             }
-            uint32_t hw[8], lw[8];
-            bool bad = false;
-#pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-              __half h0, l0, h1, l1;
-              const float a0 = __fmul_rn(__fdiv_rn(v[i], __fadd_rn(1.0f, expf(-v[i]))), v[16 + i]);
-              const float a1 = __fmul_rn(__fdiv_rn(v[i + 1], __fadd_rn(1.0f, expf(-v[i + 1]))), v[17 + i]);
-              bad |= inv::f16_overflow(a0) | inv::f16_overflow(a1);
-              inv::split_hi_lo(a0, h0, l0);
-              inv::split_hi_lo(a1, h1, l1);
-              hw[i / 2] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
-              lw[i / 2] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
-            }
-            if (bad) inv::record_status(status, INV_ERR_RANGE);
-            uint4* gh = reinterpret_cast<uint4*>(gate_hi + (int64_t)row * ld_g + f0);
-            uint4* gl = reinterpret_cast<uint4*>(gate_lo + (int64_t)row * ld_g + f0);
-            gh[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-            gh[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
-            gl[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-            gl[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
-          }
-        } else if (row < M &&
-                   INV_SPAN_IN_BOUNDS(status, col0, col0 + EPI_COLS - 1, N) &&
-                   INV_SPAN_IN_BOUNDS(status, (int64_t)row * ld_y + col0, (int64_t)row * ld_y + col0 + EPI_COLS - 1,
-                                      (int64_t)(M - 1) * ld_y + N) &&
-                   (residual == nullptr ||
-                    INV_SPAN_IN_BOUNDS(status, (int64_t)row * ld_r + col0, (int64_t)row * ld_r + col0 + EPI_COLS - 1,
-                                       (int64_t)(M - 1) * ld_r + N))) {
-          // (index checks above: column exponents, y [M][ld_y] and residual [M][ld_r], N columns used)
-          float* yr = y + (int64_t)row * ld_y + col0;
-          const float* rr = residual ? residual + (int64_t)row * ld_r + col0 : nullptr;
-#pragma unroll
-          for (int i = 0; i < EPI_COLS; i += 4) {
-            const char4 e4 = *reinterpret_cast<const char4*>(col_exp + col0 + i);
-            const int ev[4] = {e4.x, e4.y, e4.z, e4.w};
-            float o[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float t = __fadd_rn(acc_h[i + j], __fmul_rn(acc_x[i + j], 0x1p-11f));
-              o[j] = __fmul_rn(t, inv::pow2f(-ev[j]));
-            }
-            if (rr) {
-              const float4 r4 = *reinterpret_cast<const float4*>(rr + i);
-              o[0] = __fadd_rn(o[0], r4.x);
-              o[1] = __fadd_rn(o[1], r4.y);
-              o[2] = __fadd_rn(o[2], r4.z);
-              o[3] = __fadd_rn(o[3], r4.w);
-            }
-            *reinterpret_cast<float4*>(yr + i) = make_float4(o[0], o[1], o[2], o[3]);
           }
         }
+        if (ready_out != nullptr) {
+          // publish: this warp's stores of the tile, then one release add per
+          // warp; the tile is complete when all EPI_WARPS warps have added
+          __threadfence();
+          __syncwarp();
+          if (lane == 0 && INV_IN_BOUNDS(status, (int64_t)mt * (N / BN) + nt, (int64_t)tiles_m * (N / BN)))
+            inv::red_release_gpu_add(ready_out + (int64_t)mt * (N / BN) + nt, 1);
+        }
       }
-      if (ready_out != nullptr) {
-        // publish: this warp's stores of the tile, then one release add per
-        // warp; the tile is complete when all EPI_WARPS warps have added
-        __threadfence();
-        __syncwarp();
-        if (lane == 0 && INV_IN_BOUNDS(status, (int64_t)mt * (N / BN) + nt, (int64_t)tiles_m * (N / BN)))
-          inv::red_release_gpu_add(ready_out + (int64_t)mt * (N / BN) + nt, 1);
+    } else {
+      const int quarter = warp & 3;
+      const int half = (warp - 2) >> 2;
+      constexpr int QC = BN / 4;
+      const auto tcol = [half](int c) { return c < QC ? half * QC + c : 2 * QC + half * QC + (c - QC); };
+      if (ai.zero_a != nullptr)  // counters of a later kernel, cleared here (any CTA, any order)
+        for (int64_t i = (int64_t)blockIdx.x * (THREADS - 64) + (threadIdx.x - 64); i < ai.n_a;
+             i += (int64_t)gridDim.x * (THREADS - 64))
+          if (INV_IN_BOUNDS(status, i, ai.n_a)) ai.zero_a[i] = 0;
+      uint32_t g = 0;
+      for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        const int nt = tile / tiles_m, mt = tile - nt * tiles_m;
+        float acc_h[EPI_COLS], acc_x[EPI_COLS];
+#pragma unroll
+        for (int i = 0; i < EPI_COLS; ++i) acc_h[i] = acc_x[i] = 0.0f;
+        for (int grp = 0; grp < ngroups; ++grp, ++g) {
+          const uint32_t buf = g & 1u, tph = (g >> 1) & 1u;
+          int okw = 1;
+          if (lane == 0) okw = inv::mbar_wait(&sm.tfull[buf], tph, wait_ns, abort_flag, status) ? 1 : 0;
+          okw = __shfl_sync(0xffffffffu, okw, 0);  // keep the warp converged for tcgen05.ld
+          // with the fused attention inputs the two warps of a row block meet
+          // at a barrier later on: they leave (after a failed wait) together
+          okw = pair_all(okw != 0, 1 + quarter) ? 1 : 0;
+          if (!okw) goto epi_done;
+          inv::tc_fence_after();
+          const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * ACC_COLS;
+#pragma unroll
+          for (int c = 0; c < EPI_COLS; c += 16) {
+            uint32_t rh[16], rx[16];
+            inv::tmem_ld_32x16(ta + tcol(c), rh);
+            inv::tmem_ld_32x16(ta + BN + tcol(c), rx);
+            inv::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              acc_h[c + i] = __fadd_rn(acc_h[c + i], __uint_as_float(rh[i]));
+              acc_x[c + i] = __fadd_rn(acc_x[c + i], __uint_as_float(rx[i]));
+            }
+          }
+          inv::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) inv::mbar_arrive(&sm.tempty[buf]);
+        }
+        {
+          const int row = mt * BM + quarter * 32 + lane;
+          const int col0 = nt * BN;  // first column of the tile
+          // y = (hh + 2^-11 cross) 2^-e_n per column, into acc_h
+          auto scale_cols = [&]() {
+#pragma unroll
+            for (int c = 0; c < EPI_COLS; c += 4) {
+              const char4 e4 = *reinterpret_cast<const char4*>(col_exp + col0 + tcol(c));
+              const int ev[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                acc_h[c + j] = __fmul_rn(__fadd_rn(acc_h[c + j], __fmul_rn(acc_x[c + j], 0x1p-11f)), inv::pow2f(-ev[j]));
+            }
+          };
+          {
+            // Fused attention inputs (one 128-wide head per tile): rotary
+            // embedding of query and key heads, then query heads to q_out and
+            // key/value heads INT16-quantised into the cache at (slot, pos) of
+            // the row; len = pos + 1.  Same arithmetic, in the same order, as
+            // the rotary and quantiser definitions on the stored fp32 values.
+            const bool in_row = row < M;
+            int sl = 0, p = 0;
+            bool ok = false;
+            if (in_row) {
+              sl = ai.slot[row];
+              p = ai.pos[row];
+              ok = sl >= 0 && sl < ai.cache.n_slots && p >= 0 && p < ai.cache.max_len && p < ai.max_pos;
+              if (nt == 0 && half == 0) {
+                if (INV_IN_BOUNDS(status, row, M)) ai.len_out[row] = ok ? p + 1 : 0;
+                if (!ok) inv::record_status(status, INV_ERR_INVALID_ARG);
+              }
+            }
+            const int Hkv = ai.cache.n_kv_heads;
+            const bool is_q = nt < ai.Hq, is_k = !is_q && nt < ai.Hq + Hkv;
+            if (ok && (!INV_IN_BOUNDS(status, col0 + BN - 1, N) ||
+                       !INV_SPAN_IN_BOUNDS(status, (int64_t)p * 64, (int64_t)p * 64 + 63, (int64_t)ai.max_pos * 64)))
+              ok = false;
+            if (ok) {
+              scale_cols();
+              if (is_q || is_k) {
+                // rotate-half: columns j and j + 64 (local c and c + QC), frequency j
+                const float* cs = ai.rope_cos + (int64_t)p * 64 + half * QC;
+                const float* sn = ai.rope_sin + (int64_t)p * 64 + half * QC;
+#pragma unroll
+                for (int c = 0; c < QC; c += 4) {
+                  const float4 c4 = *reinterpret_cast<const float4*>(cs + c);
+                  const float4 s4 = *reinterpret_cast<const float4*>(sn + c);
+                  const float cv[4] = {c4.x, c4.y, c4.z, c4.w}, sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) {
+                    const float lo = acc_h[c + j], hi = acc_h[QC + c + j];
+                    acc_h[c + j] = __fsub_rn(__fmul_rn(lo, cv[j]), __fmul_rn(hi, sv[j]));
+                    acc_h[QC + c + j] = __fadd_rn(__fmul_rn(hi, cv[j]), __fmul_rn(lo, sv[j]));
+                  }
+                }
+              }
+            }
+            if (is_q) {
+              const int64_t qb = ((int64_t)row * ai.Hq + nt) * 128;
+              if (ok && INV_SPAN_IN_BOUNDS(status, qb, qb + 127, (int64_t)M * ai.Hq * 128)) {
+#pragma unroll
+                for (int c = 0; c < EPI_COLS; c += 4)
+                  *reinterpret_cast<float4*>(ai.q_out + qb + tcol(c)) =
+                      make_float4(acc_h[c], acc_h[c + 1], acc_h[c + 2], acc_h[c + 3]);
+              }
+            } else {
+              // max |x| over the row's 128 values: this thread's EPI_COLS, then
+              // the partner warp's (same rows, other half) through shared memory;
+              // NaN is ignored by fmaxf as in the quantiser's definition
+              float m = fabsf(acc_h[0]);
+#pragma unroll
+              for (int c = 1; c < EPI_COLS; ++c) m = fmaxf(m, fabsf(acc_h[c]));
+              // exchange with the partner warp (same rows, other half); the
+              // second barrier keeps the next tile's write after both reads
+              float* rm = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(&sm) + sizeof(GemmSmem));
+              rm[half * BM + quarter * 32 + lane] = m;
+              asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");  // the warp pair of these rows
+              m = fmaxf(m, rm[(half ^ 1) * BM + quarter * 32 + lane]);
+              asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
+              const int h = is_k ? nt - ai.Hq : nt - ai.Hq - Hkv;
+              const int64_t rowi = ((int64_t)sl * Hkv + h) * ai.cache.max_len + p;
+              if (ok && INV_IN_BOUNDS(status, rowi, (int64_t)ai.cache.n_slots * Hkv * ai.cache.max_len)) {
+                const float sc = __fdiv_rn(m, 32767.0f);
+                int16_t* codes = (is_k ? ai.cache.k : ai.cache.v) + rowi * 128;
+#pragma unroll
+                for (int c = 0; c < EPI_COLS; c += 8) {
+                  uint32_t w4[4];
+#pragma unroll
+                  for (int j = 0; j < 8; j += 2) {
+                    int q2[2] = {0, 0};
+                    if (sc != 0.0f)
+#pragma unroll
+                      for (int u = 0; u < 2; ++u) {
+                        const int t = __float2int_rn(__fdiv_rn(acc_h[c + j + u], sc));  // round half to even
+                        q2[u] = t > 32767 ? 32767 : (t < -32767 ? -32767 : t);
+                      }
+                    w4[j / 2] = (uint32_t)(uint16_t)q2[0] | ((uint32_t)(uint16_t)q2[1] << 16);
+                  }
+                  *reinterpret_cast<uint4*>(codes + tcol(c)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+                if (half == 0) (is_k ? ai.cache.k_scale : ai.cache.v_scale)[rowi] = sc;
+              }
+            }
+          }
+        }
+        if (ready_out != nullptr) {
+          // publish: this warp's stores of the tile, then one release add per
+          // warp; the tile is complete when all EPI_WARPS warps have added
+          __threadfence();
+          __syncwarp();
+          if (lane == 0 && INV_IN_BOUNDS(status, (int64_t)mt * (N / BN) + nt, (int64_t)tiles_m * (N / BN)))
+            inv::red_release_gpu_add(ready_out + (int64_t)mt * (N / BN) + nt, 1);
+        }
       }
     }
   epi_done:;
@@ -360,12 +549,33 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (ready_in != nullptr) inv::grid_wait_prerequisites();
 }
 
-// One launch of the BN-wide kernel (arguments validated by the caller).
 template <int BN>
+__global__ void __launch_bounds__(THREADS, 1)
+    comp_gemm_kernel(const __grid_constant__ CUtensorMap tm_ahi, const __grid_constant__ CUtensorMap tm_alo,
+                     const __grid_constant__ CUtensorMap tm_w, const int8_t* __restrict__ col_exp, float* y,
+                     int64_t ld_y, const float* residual, int64_t ld_r, __half* gate_hi, __half* gate_lo,
+                     int64_t ld_g, int M, int N, int K, int box_rows, int a_stride, int n_stages, int* ready_out,
+                     const int* ready_in, int* status, long long wait_ns) {
+  gemm_body<BN, false>(tm_ahi, tm_alo, tm_w, col_exp, y, ld_y, residual, ld_r, gate_hi, gate_lo, ld_g, M, N, K,
+                       box_rows, a_stride, n_stages, ready_out, ready_in, status, wait_ns, inv::AttnInputs{});
+}
+
+template <int BN>
+__global__ void __launch_bounds__(THREADS, 1)
+    qkv_attn_kernel(const __grid_constant__ CUtensorMap tm_ahi, const __grid_constant__ CUtensorMap tm_alo,
+                    const __grid_constant__ CUtensorMap tm_w, const int8_t* __restrict__ col_exp, int M, int N, int K,
+                    int box_rows, int a_stride, int n_stages, int* status, long long wait_ns,
+                    const inv::AttnInputs ai) {
+  gemm_body<BN, true>(tm_ahi, tm_alo, tm_w, col_exp, nullptr, 0, nullptr, 0, nullptr, nullptr, 0, M, N, K, box_rows,
+                      a_stride, n_stages, nullptr, nullptr, status, wait_ns, ai);
+}
+
+// One launch of the BN-wide kernel (arguments validated by the caller).
+template <int BN, bool kAttnIn>
 int launch_tiles(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a, const uint16_t* w_packed,
                  const int8_t* col_exp, int N, float* y, int64_t ld_y, const float* residual, int64_t ld_r,
                  uint16_t* gate_hi, uint16_t* gate_lo, int64_t ld_g, int* ready_out, const int* ready_in,
-                 cudaStream_t s, long long wait_ns) {
+                 cudaStream_t s, long long wait_ns, const inv::AttnInputs& ai) {
   static bool attr_set[64] = {};
   // A rows per load: the whole 128-row tile, or only round_up(M, 8) when M < 128
   const int box_rows = M < BM ? (int)((M + 7) / 8 * 8) : BM;
@@ -389,9 +599,12 @@ int launch_tiles(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, i
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(comp_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
-        cudaSuccess)
-      return INV_ERR_CUDA;
+    const cudaError_t ea =
+        kAttnIn ? cudaFuncSetAttribute(qkv_attn_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem_bytes<true>())
+                : cudaFuncSetAttribute(comp_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem_bytes<false>());
+    if (ea != cudaSuccess) return INV_ERR_CUDA;
     attr_set[dev] = true;
   }
   const int64_t tiles = ((M + BM - 1) / BM) * (N / BN);
@@ -402,17 +615,21 @@ int launch_tiles(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, i
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(grid);
   lc.blockDim = dim3(THREADS);
-  lc.dynamicSmemBytes = kSmemBytes;
+  lc.dynamicSmemBytes = smem_bytes<kAttnIn>();
   lc.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = ready_in != nullptr ? 1 : 0;
-  const cudaError_t e = cudaLaunchKernelEx(&lc, comp_gemm_kernel<BN>, ta, tl, tw, col_exp, y, ld_y, residual, ld_r,
-                                           reinterpret_cast<__half*>(gate_hi), reinterpret_cast<__half*>(gate_lo),
-                                           ld_g, (int)M, N, K, box_rows, a_stride, n_stages, ready_out, ready_in,
-                                           inv::status_ptr(), wait_ns < 0 ? inv::wait_limit_ns() : wait_ns);
+  const long long wl = wait_ns < 0 ? inv::wait_limit_ns() : wait_ns;
+  const cudaError_t e =
+      kAttnIn ? cudaLaunchKernelEx(&lc, qkv_attn_kernel<BN>, ta, tl, tw, col_exp, (int)M, N, K, box_rows, a_stride,
+                                   n_stages, inv::status_ptr(), wl, ai)
+              : cudaLaunchKernelEx(&lc, comp_gemm_kernel<BN>, ta, tl, tw, col_exp, y, ld_y, residual, ld_r,
+                                   reinterpret_cast<__half*>(gate_hi), reinterpret_cast<__half*>(gate_lo), ld_g,
+                                   (int)M, N, K, box_rows, a_stride, n_stages, ready_out, ready_in,
+                                   inv::status_ptr(), wl);
   if (e != cudaSuccess) return INV_ERR_CUDA;
   INV_CHECK_LAUNCH();
   return INV_OK;
@@ -439,19 +656,19 @@ int launch_comp_gemm_ex(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, i
                         const float* residual, int64_t ld_r, uint16_t* gate_hi, uint16_t* gate_lo, int64_t ld_g,
                         int* ready_out, const int* ready_in, cudaStream_t s, long long wait_ns) {
   if (M == 0) return INV_OK;
-  switch (gemm_panel_width(N)) {
-    case 128:
-      return launch_tiles<128>(a_hi, a_lo, M, K, ld_a, w_packed, col_exp, N, y, ld_y, residual, ld_r, gate_hi, gate_lo,
-                               ld_g, ready_out, ready_in, s, wait_ns);
-    case 64:
-      return launch_tiles<64>(a_hi, a_lo, M, K, ld_a, w_packed, col_exp, N, y, ld_y, residual, ld_r, gate_hi, gate_lo,
-                              ld_g, ready_out, ready_in, s, wait_ns);
-    case 32:
-      return launch_tiles<32>(a_hi, a_lo, M, K, ld_a, w_packed, col_exp, N, y, ld_y, residual, ld_r, gate_hi, gate_lo,
-                              ld_g, ready_out, ready_in, s, wait_ns);
-    default:
-      return INV_ERR_UNSUPPORTED_SHAPE;
-  }
+  if (gemm_panel_width(N) != INV_GEMM_BN) return INV_ERR_UNSUPPORTED_SHAPE;
+  return launch_tiles<INV_GEMM_BN, false>(a_hi, a_lo, M, K, ld_a, w_packed, col_exp, N, y, ld_y, residual, ld_r, gate_hi,
+                                   gate_lo, ld_g, ready_out, ready_in, s, wait_ns, AttnInputs{});
+}
+
+int launch_qkv_attn_inputs(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
+                           const uint16_t* w_packed, const int8_t* col_exp, int N, const AttnInputs& ai,
+                           cudaStream_t s) {
+  if (M == 0) return INV_OK;
+  if (gemm_panel_width(N) != INV_GEMM_BN || N != (ai.Hq + 2 * ai.cache.n_kv_heads) * INV_HEAD_DIM)
+    return INV_ERR_UNSUPPORTED_SHAPE;
+  return launch_tiles<INV_GEMM_BN, true>(a_hi, a_lo, M, K, ld_a, w_packed, col_exp, N, nullptr, 0, nullptr, 0, nullptr,
+                                   nullptr, 0, nullptr, nullptr, s, -1, ai);
 }
 
 }  // namespace inv

@@ -14,7 +14,6 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct LayerWs {
   uint16_t *h_hi, *h_lo;
-  float* qkv;
   float* q_rot;
   int32_t* lens;
   int32_t* rows_slot;  // prefill_layer: per-row slot / position arrays
@@ -38,10 +37,8 @@ LayerWs carve(const inv_layer_config& c, int B, int mlb, uint8_t* base) {
     return p;
   };
   const size_t H = c.hidden, F = c.ffn, QD = (size_t)c.n_heads * 128;
-  const size_t NQKV = (size_t)(c.n_heads + 2 * c.n_kv_heads) * 128;
   w.h_hi = reinterpret_cast<uint16_t*>(take(B * H * 2));
   w.h_lo = reinterpret_cast<uint16_t*>(take(B * H * 2));
-  w.qkv = reinterpret_cast<float*>(take(B * NQKV * 4));
   w.q_rot = reinterpret_cast<float*>(take(B * QD * 4));
   w.lens = reinterpret_cast<int32_t*>(take(B * 4));
   w.rows_slot = reinterpret_cast<int32_t*>(take(B * 4));
@@ -112,32 +109,44 @@ int run_layer(const inv_layer_config* cfg, const inv_layer_weights* w, const inv
   } while (0)
   // 1. h = rmsnorm(x) -> hi/lo
   INV_TRACED(0, inv::launch_rmsnorm(x_in, w->g_attn, B, H, cfg->eps, nullptr, ws.h_hi, ws.h_lo, s));
-  // 2. qkv = h W_qkv
-  INV_TRACED(1, inv::launch_comp_gemm(ws.h_hi, ws.h_lo, B, H, H, w->w_qkv, w->e_qkv, NQKV, ws.qkv, NQKV, nullptr, 0, s));
-  // 3. rotary embedding of q and k; k, v -> INT16 cache; len = pos + 1
-  //    (it also clears the gate/up tile counters of this layer; the previous
-  //    layer has finished with them)
-  INV_TRACED(2, inv::launch_rope_quant(ws.qkv, B, Hq, *cache, slot, pos, w->rope_cos, w->rope_sin, cfg->max_pos,
-                                       ws.q_rot, ws.lens, ws.ready, (int64_t)(inv::gemm_ready_bytes(B, 2 * F) / 4), s));
-  // 4-5. fixed-split attention + ordered combine -> o hi/lo (kernels 3 and 4)
+  // 2. [q | k | v] = h W_qkv with, in the GEMM's epilogue, the rotary
+  //    embedding of q and k, k and v INT16-quantised into the cache, q to
+  //    q_rot, len = pos + 1 (and the gate/up tile counters of this layer
+  //    cleared; the previous layer has finished with them)
+  {
+    inv::AttnInputs ai;
+    ai.slot = slot;
+    ai.pos = pos;
+    ai.rope_cos = w->rope_cos;
+    ai.rope_sin = w->rope_sin;
+    ai.max_pos = cfg->max_pos;
+    ai.q_out = ws.q_rot;
+    ai.Hq = Hq;
+    ai.cache = *cache;
+    ai.len_out = ws.lens;
+    ai.zero_a = ws.ready;
+    ai.n_a = (int64_t)(inv::gemm_ready_bytes(B, 2 * F) / 4);
+    INV_TRACED(1, inv::launch_qkv_attn_inputs(ws.h_hi, ws.h_lo, B, H, H, w->w_qkv, w->e_qkv, NQKV, ai, s));
+  }
+  // 3-4. fixed-split attention + ordered combine -> o hi/lo (kernels 2 and 3)
   if (prefill_slot < 0) {
     INV_TRY(inv::launch_attention(ws.q_rot, B, Hq, *cache, slot, ws.lens, mlb, cfg->softmax_scale, ws.o, ws.o_hi,
-                                  ws.o_lo, ws.attn, s, 3));
+                                  ws.o_lo, ws.attn, s, 2));
   } else {
     INV_TRY(inv::launch_attention_prefill(ws.q_rot, B, Hq, *cache, prefill_slot, prefill_pos0, ws.lens, mlb,
-                                          cfg->softmax_scale, ws.o, ws.o_hi, ws.o_lo, ws.attn, s, 3));
+                                          cfg->softmax_scale, ws.o, ws.o_hi, ws.o_lo, ws.attn, s, 2));
   }
-  // 6. x1 = x + o W_o
-  INV_TRACED(5, inv::launch_comp_gemm(ws.o_hi, ws.o_lo, B, QD, QD, w->w_o, w->e_o, H, ws.x1, H, x_in, H, s));
-  // 7. h2 = rmsnorm(x1) -> hi/lo
-  INV_TRACED(6, inv::launch_rmsnorm(ws.x1, w->g_mlp, B, H, cfg->eps, nullptr, ws.h2_hi, ws.h2_lo, s));
-  // 8-9. [gate | up] = h2 W_gu with the SwiGLU a = silu(gate) * up fused in the epilogue -> hi/lo
-  // 10. out = x1 + a W_down.  The down GEMM starts while the gate/up GEMM's
+  // 5. x1 = x + o W_o
+  INV_TRACED(4, inv::launch_comp_gemm(ws.o_hi, ws.o_lo, B, QD, QD, w->w_o, w->e_o, H, ws.x1, H, x_in, H, s));
+  // 6. h2 = rmsnorm(x1) -> hi/lo
+  INV_TRACED(5, inv::launch_rmsnorm(ws.x1, w->g_mlp, B, H, cfg->eps, nullptr, ws.h2_hi, ws.h2_lo, s));
+  // 7. [gate | up] = h2 W_gu with the SwiGLU a = silu(gate) * up fused in the epilogue -> hi/lo
+  // 8. out = x1 + a W_down.  The down GEMM starts while the gate/up GEMM's
   // last tiles (a partial wave) run, loading each 64-column K block of a as
   // soon as the gate/up tile that stores it has published it.
-  INV_TRACED(7, inv::launch_comp_gemm_ex(ws.h2_hi, ws.h2_lo, B, H, H, w->w_gu, w->e_gu, 2 * F, nullptr, 0, nullptr, 0,
+  INV_TRACED(6, inv::launch_comp_gemm_ex(ws.h2_hi, ws.h2_lo, B, H, H, w->w_gu, w->e_gu, 2 * F, nullptr, 0, nullptr, 0,
                                          ws.a_hi, ws.a_lo, F, ws.ready, nullptr, s));
-  INV_TRACED(8, inv::launch_comp_gemm_ex(ws.a_hi, ws.a_lo, B, F, F, w->w_down, w->e_down, H, x_out, H, ws.x1, H,
+  INV_TRACED(7, inv::launch_comp_gemm_ex(ws.a_hi, ws.a_lo, B, F, F, w->w_down, w->e_down, H, x_out, H, ws.x1, H,
                                          nullptr, nullptr, 0, nullptr, ws.ready, s));
 #undef INV_TRACED
   return INV_OK;

@@ -1,7 +1,8 @@
 // Bandwidth-bound kernels of the decode step: the binary16 hi/lo split, the
 // offline weight packing, batch-invariant RMSNorm, the INT16 KV quantiser, and
-// the per-row glue of the layer (rotary embedding + quantisation, embedding
-// gather, greedy argmax).  All use 128-bit coalesced accesses where
+// the per-row glue of the stack (rotary tables, embedding gather, greedy
+// argmax).  The rotary embedding itself and the quantisation of a layer's new
+// keys and values run in the QKV GEMM's epilogue (comp_gemm.cu).  All use 128-bit coalesced accesses where
 // the layout allows and fixed, shape-independent reduction orders.
 #include "common.cuh"
 #include "internal.h"
@@ -309,78 +310,6 @@ __global__ void kv_quant_kernel(const float* __restrict__ x, int T, int64_t ld_x
   quant_store_row(v, codes, scale, lane);
 }
 
-// Rotary embedding (rotate-half, pairs (i, i+64)) of one 128-wide head held as
-// one float4 per lane; the partner of lane l is lane l ^ 16.
-__device__ __forceinline__ float4 rope_row(float4 v, const float* __restrict__ cs, const float* __restrict__ sn,
-                                           int lane) {
-  float4 p;
-  p.x = __shfl_xor_sync(0xffffffffu, v.x, 16);
-  p.y = __shfl_xor_sync(0xffffffffu, v.y, 16);
-  p.z = __shfl_xor_sync(0xffffffffu, v.z, 16);
-  p.w = __shfl_xor_sync(0xffffffffu, v.w, 16);
-  const int i0 = (lane & 15) * 4;  // frequency index of v.x
-  const float4 c = *reinterpret_cast<const float4*>(cs + i0);
-  const float4 s = *reinterpret_cast<const float4*>(sn + i0);
-  float4 o;
-  if (lane < 16) {  // first half: x_i cos - x_{i+64} sin
-    o.x = __fsub_rn(__fmul_rn(v.x, c.x), __fmul_rn(p.x, s.x));
-    o.y = __fsub_rn(__fmul_rn(v.y, c.y), __fmul_rn(p.y, s.y));
-    o.z = __fsub_rn(__fmul_rn(v.z, c.z), __fmul_rn(p.z, s.z));
-    o.w = __fsub_rn(__fmul_rn(v.w, c.w), __fmul_rn(p.w, s.w));
-  } else {          // second half: x_{i+64} cos + x_i sin
-    o.x = __fadd_rn(__fmul_rn(v.x, c.x), __fmul_rn(p.x, s.x));
-    o.y = __fadd_rn(__fmul_rn(v.y, c.y), __fmul_rn(p.y, s.y));
-    o.z = __fadd_rn(__fmul_rn(v.z, c.z), __fmul_rn(p.z, s.z));
-    o.w = __fadd_rn(__fmul_rn(v.w, c.w), __fmul_rn(p.w, s.w));
-  }
-  return o;
-}
-
-// Layer glue: per (token, head index) warp over the fused qkv rows.  Query
-// heads are rotated and written to q_out; key heads rotated then quantised;
-// value heads quantised.  Also writes len[t] = pos[t] + 1.
-__global__ void rope_quant_kernel(const float* __restrict__ qkv, int T, int Hq, inv_kv_cache c,
-                                  const int32_t* __restrict__ slot, const int32_t* __restrict__ pos,
-                                  const float* __restrict__ rope_cos, const float* __restrict__ rope_sin, int max_pos,
-                                  float* __restrict__ q_out, int32_t* __restrict__ len_out, int* __restrict__ zero_a,
-                                  int64_t n_a, int* status) {
-  {
-    const int64_t t0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x, stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = t0; i < n_a; i += stride)
-      if (INV_IN_BOUNDS(status, i, n_a)) zero_a[i] = 0;
-  }
-  const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const int Hkv = c.n_kv_heads;
-  const int nh = Hq + 2 * Hkv;
-  if (warp >= (int64_t)T * nh) return;
-  const int t = (int)(warp / nh), hi = (int)(warp - (int64_t)t * nh);
-  const int sl = slot[t], p = pos[t];
-  const bool ok = sl >= 0 && sl < c.n_slots && p >= 0 && p < c.max_len && p < max_pos;
-  if (hi == 0 && lane == 0 && INV_IN_BOUNDS(status, t, T)) len_out[t] = ok ? p + 1 : 0;
-  if (!ok) {
-    if (lane == 0 && hi == 0) record_status(status, INV_ERR_INVALID_ARG);
-    return;
-  }
-  const int64_t iq = (int64_t)t * nh * 128 + (int64_t)hi * 128;
-  if (!INV_SPAN_IN_BOUNDS(status, iq, iq + 127, (int64_t)T * nh * 128) ||
-      !INV_SPAN_IN_BOUNDS(status, (int64_t)p * 64, (int64_t)p * 64 + 63, (int64_t)max_pos * 64))
-    return;
-  float4 v = reinterpret_cast<const float4*>(qkv + iq)[lane];
-  if (hi < Hq + Hkv) v = rope_row(v, rope_cos + (int64_t)p * 64, rope_sin + (int64_t)p * 64, lane);
-  if (hi < Hq) {
-    const int64_t io = ((int64_t)t * Hq + hi) * 128;
-    if (INV_SPAN_IN_BOUNDS(status, io, io + 127, (int64_t)T * Hq * 128))
-      reinterpret_cast<float4*>(q_out + io)[lane] = v;
-    return;
-  }
-  const bool is_k = hi < Hq + Hkv;
-  const int h = is_k ? hi - Hq : hi - Hq - Hkv;
-  const int64_t rowi = ((int64_t)sl * Hkv + h) * c.max_len + p;
-  if (!INV_IN_BOUNDS(status, rowi, (int64_t)c.n_slots * Hkv * c.max_len)) return;
-  quant_store_row(v, (is_k ? c.k : c.v) + rowi * 128, (is_k ? c.k_scale : c.v_scale) + rowi, lane);
-}
-
 __global__ void embed_kernel(const float* __restrict__ table, int vocab, int hidden, const int32_t* __restrict__ ids,
                              int B, float* __restrict__ x, int* status) {
   const int b = blockIdx.x;
@@ -464,19 +393,6 @@ int launch_rmsnorm(const float* x, const float* gamma, int64_t rows, int hidden,
     rmsnorm_reg_kernel<8><<<(unsigned)rows, kNormThreads, 0, s>>>(x, gamma, hidden, eps, y, h, l, status_ptr());
   else
     rmsnorm_kernel<<<(unsigned)rows, kNormThreads, 0, s>>>(x, gamma, hidden, eps, y, h, l, status_ptr());
-  INV_CHECK_LAUNCH();
-  return INV_OK;
-}
-
-int launch_rope_quant(const float* qkv, int T, int Hq, const inv_kv_cache& c, const int32_t* slot,
-                      const int32_t* pos, const float* rope_cos, const float* rope_sin, int max_pos, float* q_out,
-                      int32_t* len_out, int* zero_a, int64_t n_a, cudaStream_t s) {
-  if (T == 0) return INV_OK;
-  const int64_t warps = (int64_t)T * (Hq + 2 * c.n_kv_heads);
-  const int threads = 256;
-  const int64_t blocks = (warps * 32 + threads - 1) / threads;
-  rope_quant_kernel<<<(unsigned)blocks, threads, 0, s>>>(qkv, T, Hq, c, slot, pos, rope_cos, rope_sin, max_pos, q_out,
-                                                        len_out, zero_a, zero_a ? n_a : 0, status_ptr());
   INV_CHECK_LAUNCH();
   return INV_OK;
 }

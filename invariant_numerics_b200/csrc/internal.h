@@ -12,11 +12,26 @@ namespace inv {
 int launch_rmsnorm(const float* x, const float* gamma, int64_t rows, int hidden, float eps, float* y,
                    uint16_t* yh, uint16_t* yl, cudaStream_t s);
 
-// Also sets zero_a[0 .. n_a) to zero (counters a later kernel of the layer
-// needs cleared; may be null).
-int launch_rope_quant(const float* qkv, int T, int Hq, const inv_kv_cache& c, const int32_t* slot,
-                      const int32_t* pos, const float* rope_cos, const float* rope_sin, int max_pos, float* q_out,
-                      int32_t* len_out, int* zero_a, int64_t n_a, cudaStream_t s);
+// Where the QKV GEMM's epilogue puts the attention inputs of its M rows
+// (row t at position pos[t] of sequence slot[t]): query heads rotated into
+// q_out [M][Hq][128], key heads rotated and value heads as they are,
+// INT16-quantised into the cache; len_out[t] = pos[t] + 1 (0 and
+// INV_ERR_INVALID_ARG for a slot or position out of range, whose row is then
+// skipped).  zero_a[0 .. n_a) is cleared on the way (counters a later kernel
+// of the layer needs zero; may be null).  q_out == nullptr: no fusion.
+struct AttnInputs {
+  const int32_t* slot = nullptr;
+  const int32_t* pos = nullptr;
+  const float* rope_cos = nullptr;  // [max_pos][64]
+  const float* rope_sin = nullptr;
+  int max_pos = 0;
+  float* q_out = nullptr;
+  int Hq = 0;
+  inv_kv_cache cache = {};
+  int32_t* len_out = nullptr;
+  int* zero_a = nullptr;
+  int64_t n_a = 0;
+};
 
 
 // Panel width (output columns per GEMM tile and per packed panel) of a weight
@@ -43,6 +58,12 @@ int launch_comp_gemm_ex(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, i
                         const uint16_t* w_packed, const int8_t* col_exp, int N, float* y, int64_t ld_y,
                         const float* residual, int64_t ld_r, uint16_t* gate_hi, uint16_t* gate_lo, int64_t ld_g,
                         int* ready_out, const int* ready_in, cudaStream_t s, long long wait_ns = -1);
+// The QKV projection with the rotary embedding and the KV quantiser in its
+// epilogue (one 128-wide head per tile; N = (Hq + 2 Hkv) 128): writes the
+// attention inputs described by `ai` instead of the GEMM's output.
+int launch_qkv_attn_inputs(const uint16_t* a_hi, const uint16_t* a_lo, int64_t M, int K, int64_t ld_a,
+                           const uint16_t* w_packed, const int8_t* col_exp, int N, const AttnInputs& ai,
+                           cudaStream_t s);
 // Bytes of the ready array of a producer GEMM with M rows and N columns.
 inline size_t gemm_ready_bytes(int64_t M, int N) { return (size_t)((M + 127) / 128) * (size_t)(N / 128) * 4; }
 

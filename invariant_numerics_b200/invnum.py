@@ -165,8 +165,8 @@ def inv_selftest_bounds(buf, n_declared: int, n_written: int, stream=None) -> No
     _check("inv_selftest_bounds", lib.inv_selftest_bounds(_ptr(buf), int(n_declared), int(n_written), _stream(stream)))
 
 
-DECODE_LAYER_KERNELS = 9
-DECODE_LAYER_KERNEL_NAMES = ("rmsnorm_attn", "gemm_qkv", "rope_quant", "attn_split", "attn_combine", "gemm_o",
+DECODE_LAYER_KERNELS = 8
+DECODE_LAYER_KERNEL_NAMES = ("rmsnorm_attn", "gemm_qkv_rope_quant", "attn_split", "attn_combine", "gemm_o",
                              "rmsnorm_mlp", "gemm_gate_up_swiglu", "gemm_down")
 
 
