@@ -69,8 +69,8 @@ constexpr size_t kDecodeSmem = sizeof(DecodeSmem) + 1024;
 // rows at a time of the block (every unpacked K/V fragment feeds PF_R rows'
 // MMAs), so one SM keeps PF_GROUPS x PF_R rows in flight on the same resident
 // K and V.
-constexpr int PF_GROUPS = 4;
-constexpr int PF_R = 2;
+constexpr int PF_GROUPS = 3;
+constexpr int PF_R = 3;
 constexpr int PF_THREADS = PF_GROUPS * THREADS;
 
 struct __align__(1024) PrefillSmem {
@@ -145,7 +145,7 @@ struct RowSet {
 };
 
 // R query rows of one split: the whole per-row computation shared by the
-// decode (R = 1) and prefill (R = 2) kernels.  Each unpacked K or V fragment
+// decode (R = 1) and prefill (R = PF_R) kernels.  Each unpacked K or V fragment
 // feeds the MMAs of all R rows, and every row's accumulators receive exactly
 // the MMAs, in exactly the order, that they receive with R = 1 (an m-tile
 // beyond a row's n is skipped for that row), so a (row, split) gives the same
@@ -588,7 +588,7 @@ __global__ void __launch_bounds__(THREADS, 3)
 // split_rows -- the decode kernel's per-row code, with the same thread-to-data
 // mapping inside its 128-thread group -- on them, PF_GROUPS x PF_R rows at a
 // time.
-constexpr int ROWS_PER_CTA = 64;
+constexpr int ROWS_PER_CTA = 72;  // a multiple of PF_GROUPS x PF_R
 
 __global__ void __launch_bounds__(PF_THREADS, 1)
     attn_prefill_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
