@@ -125,3 +125,28 @@ def test_prefill_layer_bit_identical_to_decode_layer(inv):
     assert torch.equal(a.k, b.k) and torch.equal(a.v, b.v)
     assert torch.equal(a.k_scale, b.k_scale) and torch.equal(a.v_scale, b.v_scale)
     assert status() == inv.INV_OK
+
+
+def test_layer_rows_with_bad_slot_or_position_are_reported_and_skipped(inv):
+    """A row whose slot or position is out of range (checked where the QKV
+    GEMM's epilogue writes the cache) records INV_ERR_INVALID_ARG and writes
+    nothing; the other rows of the batch get the bits they get without it."""
+    p, cfg, w = make_layer(inv, **SMALL)
+    H = SMALL["H"]
+    caches = [inv.KVCache(n_slots=3, n_kv_heads=2, max_len=512) for _ in range(2)]
+    x0 = dev(synth.normal((20, H), seed=300))
+    for gc in caches:
+        inv.decode_layer(cfg, w, gc, x0, dev(np.zeros(20, np.int32)), dev(np.arange(20, dtype=np.int32)))
+    assert status() == inv.INV_OK
+    x = synth.normal((5, H), seed=301)
+    slot = np.array([0, 1, 7, 2, 1], np.int32)    # row 2: slot out of range
+    pos = np.array([20, 0, 0, 0, 600], np.int32)  # row 4: position past the cache
+    y_bad = inv.decode_layer(cfg, w, caches[0], dev(x), dev(slot), dev(pos))
+    assert status() == inv.INV_ERR_INVALID_ARG
+    keep = [0, 1, 3]
+    y_good = inv.decode_layer(cfg, w, caches[1], dev(x[keep]), dev(slot[keep]), dev(pos[keep]))
+    assert status() == inv.INV_OK
+    assert torch.equal(y_bad[keep].view(torch.int32), y_good.view(torch.int32))
+    for name in ("k", "v", "k_scale", "v_scale"):
+        a, b = getattr(caches[0], name), getattr(caches[1], name)
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8)), name
