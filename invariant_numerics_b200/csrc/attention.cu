@@ -466,14 +466,22 @@ __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& 
   for (int r = 0; r < R; ++r) {
     if (rows.n[r] <= 0) continue;
     const float* xr = xo + r * (4 * 4 * 128);
-    for (int idx = tid; idx < 4 * 128; idx += THREADS) {
-      const int head = idx >> 7, d = idx & 127;
-      if (head >= G) continue;
-      float v = xr[(0 * 4 + head) * 128 + d];
-      v = __fadd_rn(v, xr[(1 * 4 + head) * 128 + d]);
-      v = __fadd_rn(v, xr[(2 * 4 + head) * 128 + d]);
-      v = __fadd_rn(v, xr[(3 * 4 + head) * 128 + d]);
-      rows.out_o[r][head * head_stride_o + d] = v;
+    {
+      // thread t: head t / 32, d = 4 (t % 32) .. +3; the warps' partials are
+      // added in warp order 0, 1, 2, 3
+      const int head = tid >> 5, d = (tid & 31) * 4;
+      if (head < G) {
+        float4 v = *reinterpret_cast<const float4*>(xr + (0 * 4 + head) * 128 + d);
+#pragma unroll
+        for (int w = 1; w < 4; ++w) {
+          const float4 u = *reinterpret_cast<const float4*>(xr + (w * 4 + head) * 128 + d);
+          v.x = __fadd_rn(v.x, u.x);
+          v.y = __fadd_rn(v.y, u.y);
+          v.z = __fadd_rn(v.z, u.z);
+          v.w = __fadd_rn(v.w, u.w);
+        }
+        *reinterpret_cast<float4*>(rows.out_o[r] + head * head_stride_o + d) = v;
+      }
     }
     if (tid < G) {
       const RowScratch& sr = rs[r];
