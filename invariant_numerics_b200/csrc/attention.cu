@@ -60,7 +60,7 @@ struct __align__(1024) DecodeSmem {
   float ks[SPLIT];
   float vs[SPLIT];
   RowScratch rs;
-  uint64_t bar_k, bar_v[4];    // V: one barrier per warp (its 64 keys)
+  uint64_t bar_k, bar_q, bar_v[4];  // V: one barrier per warp (its 64 keys)
   int abort;
 };
 constexpr size_t kDecodeSmem = sizeof(DecodeSmem) + 1024;
@@ -169,13 +169,44 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
+// The B fragments of S^T = K Q^T for R rows: column g is query head g/2 of
+// the group, its hi part for even g and lo part for odd g; rows k = d.  Every
+// warp needs the same fragments, so the group splits each q value once: pair
+// p = (row r, k-step ks, i, head, c) holds d = 16 ks + 2 c + 8 i and d + 1, and
+// its hi and lo words go to lanes 4 (2 head) + c and 4 (2 head + 1) + c at
+// qfrag[((r 4 + j) 32 + lane) 4 + e] for ks 2 + i = 4 j + e, so that each lane
+// later reads its 16 words as 4 conflict-free 128-bit loads.
+template <int R>
+__device__ __forceinline__ void write_q_fragments(int tid, const RowSet<R>& rows, int G, uint32_t* qfrag,
+                                                  int* status) {
+  bool bad = false;
+#pragma unroll
+  for (int k = 0; k < 2 * R; ++k) {
+    const int r = k >> 1, rem = (tid + THREADS * k) & 255;
+    const int cc = rem & 3, head = (rem >> 2) & 3, q16 = rem >> 4;  // q16 = ks 2 + i
+    const int d = 16 * (q16 >> 1) + 2 * cc + 8 * (q16 & 1);
+    const bool valid = head < G && rows.n[r] > 0;
+    const float2 x = valid ? *reinterpret_cast<const float2*>(rows.q[r] + head * 128 + d) : make_float2(0.f, 0.f);
+    __half h0, l0, h1, l1;
+    inv::split_hi_lo(x.x, h0, l0);
+    inv::split_hi_lo(x.y, h1, l1);
+    bad |= inv::f16_overflow(x.x) | inv::f16_overflow(x.y);
+    uint32_t* dst = qfrag + ((r * 4 + (q16 >> 2)) * 32 + 8 * head + cc) * 4 + (q16 & 3);
+    dst[0] = pack_half2(h0, h1);
+    dst[16] = pack_half2(l0, l1);  // lane + 4
+  }
+  if (bad) record_status(status, INV_ERR_RANGE);
+}
+
+// kQReady: the caller has already written the rows' q fragments into qfrag
+// (write_q_fragments) and synchronised the group.
 // kLamp (R = 1 only): each score is also evaluated in low precision -- q16 .
 // code accumulated in binary16, one rounding per multiply-add, over d in
 // ascending order, the high and low code bytes in two accumulators -- and the
 // scores whose relaxed criterion 2 exp(y_lo - m_lo) |y_lo| exceeds tau (m_lo
 // the split's largest finite low-precision score; non-finite ones always)
 // keep the full-precision value; the others continue with y_lo.
-template <int R, bool kReuse, bool kLamp, class Sync, class IssueV, class WaitV>
+template <int R, bool kReuse, bool kLamp, bool kQReady, class Sync, class IssueV, class WaitV>
 __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& rows, int G, uint32_t kbase,
                                            uint32_t vbase, const float* ks, const float* vs, RowScratch* rs,
                                            float* xo, uint32_t* qfrag, float sigma, int64_t head_stride_o,
@@ -188,33 +219,13 @@ __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& 
 #pragma unroll
   for (int r = 0; r < R; ++r) n_max = max(n_max, rows.n[r]);
 
-  // B fragments of S^T = K Q^T: column g is query head g/2 of the group, its
-  // hi part for even g and lo part for odd g; rows k = d.  Every warp needs
-  // the same fragments, so the group splits each q value once: pair p =
-  // (row r, k-step ks, i, head, c) holds d = 16 ks + 2 c + 8 i and d + 1, and
-  // its hi and lo words go to lanes 4 (2 head) + c and 4 (2 head + 1) + c at
-  // qfrag[((r 4 + j) 32 + lane) 4 + e] for ks 2 + i = 4 j + e, so that each
-  // lane then reads its 16 words as 4 conflict-free 128-bit loads.
+  // B fragments of S^T = K Q^T (write_q_fragments' layout)
   uint32_t qf[R][8][2];
   {
-    bool bad = false;
-#pragma unroll
-    for (int k = 0; k < 2 * R; ++k) {
-      const int r = k >> 1, rem = (tid + THREADS * k) & 255;
-      const int cc = rem & 3, head = (rem >> 2) & 3, q16 = rem >> 4;  // q16 = ks 2 + i
-      const int d = 16 * (q16 >> 1) + 2 * cc + 8 * (q16 & 1);
-      const bool valid = head < G && rows.n[r] > 0;
-      const float2 x = valid ? *reinterpret_cast<const float2*>(rows.q[r] + head * 128 + d) : make_float2(0.f, 0.f);
-      __half h0, l0, h1, l1;
-      inv::split_hi_lo(x.x, h0, l0);
-      inv::split_hi_lo(x.y, h1, l1);
-      bad |= inv::f16_overflow(x.x) | inv::f16_overflow(x.y);
-      uint32_t* dst = qfrag + ((r * 4 + (q16 >> 2)) * 32 + 8 * head + cc) * 4 + (q16 & 3);
-      dst[0] = pack_half2(h0, h1);
-      dst[16] = pack_half2(l0, l1);  // lane + 4
+    if constexpr (!kQReady) {
+      write_q_fragments<R>(tid, rows, G, qfrag, status);
+      sync();
     }
-    if (bad) record_status(status, INV_ERR_RANGE);
-    sync();
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
@@ -540,34 +551,49 @@ __global__ void __launch_bounds__(THREADS, 3)
 
   if (tid == 0) {
     inv::mbar_init(&sm.bar_k, 1);
+    inv::mbar_init(&sm.bar_q, 1);
     for (int w = 0; w < 4; ++w) inv::mbar_init(&sm.bar_v[w], 1);
     sm.abort = 0;
     inv::fence_mbar_init();
   }
   __syncthreads();
   if (tid == 0) {
-    // q travels with K, so the scores start as soon as the codes land
-    inv::mbar_arrive_expect_tx(&sm.bar_k, nbox * 2 * BOX_BYTES + G * 128 * 4);
-    inv::bulk_load(sm.qs, q + obase * 128, (uint32_t)(G * 128 * 4), &sm.bar_k);
+    // q on its own barrier: its fragments are split while the codes land
+    inv::mbar_arrive_expect_tx(&sm.bar_q, G * 128 * 4);
+    inv::bulk_load(sm.qs, q + obase * 128, (uint32_t)(G * 128 * 4), &sm.bar_q);
+    inv::mbar_arrive_expect_tx(&sm.bar_k, nbox * 2 * BOX_BYTES);
     for (int bx = 0; bx < nbox; ++bx) {
       inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES, &tm_k, &sm.bar_k, 0, row0 + 64 * bx);
       inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES + BOX_BYTES, &tm_k, &sm.bar_k, 64, row0 + 64 * bx);
     }
   }
-  for (int j = tid; j < SPLIT; j += THREADS) {
-    sm.ks[j] = j < n ? kscale[(int64_t)row0 + j] : 0.0f;
-    sm.vs[j] = j < n ? vscale[(int64_t)row0 + j] : 0.0f;
+  // the scales go to registers first (stored after the q fragments are done)
+  constexpr int SPT = SPLIT / THREADS;
+  float ksr[SPT], vsr[SPT];
+#pragma unroll
+  for (int i = 0; i < SPT; ++i) {
+    const int j = tid + i * THREADS;
+    ksr[i] = j < n ? kscale[(int64_t)row0 + j] : 0.0f;
+    vsr[i] = j < n ? vscale[(int64_t)row0 + j] : 0.0f;
   }
-  __syncthreads();  // scales visible
-
+  const RowSet<1> rows = {{sm.qs}, {n}, {part_o + (obase * S_max + s) * 128}, {part_ml + obase * S_max + s}};
   bool ok = true;
-  if (lane == 0) ok = inv::mbar_wait(&sm.bar_k, 0, wait_ns, &sm.abort, status);
+  if (lane == 0) ok = inv::mbar_wait(&sm.bar_q, 0, wait_ns, &sm.abort, status);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (ok) write_q_fragments<1>(tid, rows, G, sm.qfrag, status);
+#pragma unroll
+  for (int i = 0; i < SPT; ++i) {
+    sm.ks[tid + i * THREADS] = ksr[i];
+    sm.vs[tid + i * THREADS] = vsr[i];
+  }
+  __syncthreads();  // scales and q fragments visible
+
+  if (lane == 0 && ok) ok = inv::mbar_wait(&sm.bar_k, 0, wait_ns, &sm.abort, status);
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 
   bool v_issued = false;
-  const RowSet<1> rows = {{sm.qs}, {n}, {part_o + (obase * S_max + s) * 128}, {part_ml + obase * S_max + s}};
   const LampArgs lamp = {tau, sm.qs, sel != nullptr ? sel + obase * sel_ld + key0 : nullptr, sel_ld};
-  split_rows<1, false, kLamp>(
+  split_rows<1, false, kLamp, true>(
       tid, []() { __syncthreads(); }, rows, G, cbase, cbase, sm.ks, sm.vs, &sm.rs,
       reinterpret_cast<float*>(sm.codes), sm.qfrag, sigma, (int64_t)S_max * 128, (int64_t)S_max, ok, status, lamp,
       [&]() {  // this warp is done with its K codes: bring its V codes into the same slot
@@ -586,7 +612,10 @@ __global__ void __launch_bounds__(THREADS, 3)
       });
   // No copy may still be landing in this CTA's shared memory when it exits
   // (only possible after a timed-out wait; immediate otherwise).
-  if (tid == 0) inv::mbar_wait(&sm.bar_k, 0, wait_ns, nullptr, status);
+  if (tid == 0) {
+    inv::mbar_wait(&sm.bar_q, 0, wait_ns, nullptr, status);
+    inv::mbar_wait(&sm.bar_k, 0, wait_ns, nullptr, status);
+  }
   if (lane == 0 && v_issued) inv::mbar_wait(&sm.bar_v[tid >> 5], 0, wait_ns, nullptr, status);
 }
 
@@ -671,7 +700,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     }
     // the q fragments of the rows use the start of the group's exchange buffer,
     // which is written only after the last V read
-    split_rows<PF_R, true, false>(gtid, group_sync, rows, G, kbase, vbase, sm.ks, sm.vs, sm.rs[grp], sm.xo[grp][0],
+    split_rows<PF_R, true, false, false>(gtid, group_sync, rows, G, kbase, vbase, sm.ks, sm.vs, sm.rs[grp], sm.xo[grp][0],
                                   reinterpret_cast<uint32_t*>(sm.xo[grp][0]),
                                   sigma, (int64_t)S_max * 128, (int64_t)S_max, ok, status, LampArgs{}, []() {},
                                   [](bool okv) { return okv; });
