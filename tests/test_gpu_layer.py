@@ -150,3 +150,29 @@ def test_layer_rows_with_bad_slot_or_position_are_reported_and_skipped(inv):
     for name in ("k", "v", "k_scale", "v_scale"):
         a, b = getattr(caches[0], name), getattr(caches[1], name)
         assert torch.equal(a.view(torch.uint8), b.view(torch.uint8)), name
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 4)])
+def test_layer_parity_other_group_sizes(inv, Hq, Hkv):
+    """G = Hq / Hkv = 1 and 2 through the whole layer (the QKV kernel's head
+    tiles map to q, k and v heads by these counts), prefill chunk then decode,
+    against the oracle."""
+    H, F = 256, 512
+    p, cfg, w = make_layer(inv, H, Hq, Hkv, F, max_pos=1024, seed=7)
+    oc = ref.KVCache.empty(2, Hkv, 512, 128)
+    gc = inv.KVCache(n_slots=2, n_kv_heads=Hkv, max_len=512)
+    steps = [
+        (np.zeros(261, np.int32), np.arange(261, dtype=np.int32)),
+        (np.array([0, 1], np.int32), np.array([261, 0], np.int32)),
+        (np.array([1, 0], np.int32), np.array([1, 262], np.int32)),
+    ]
+    for i, (slot, pos) in enumerate(steps):
+        x = synth.normal((len(slot), H), seed=200 + i)
+        if i == 0:  # the prompt chunk through prefill_layer (its own attention kernel)
+            y = inv.prefill_layer(cfg, w, gc, dev(x), 0, 0)
+        else:
+            y = inv.decode_layer(cfg, w, gc, dev(x), dev(slot), dev(pos))
+        want = ref.decode_layer(p, oc, x, slot, pos)
+        err = rowwise_err(host(y), want)
+        assert err.max() <= TOL, (i, err.max())
+    assert status() == inv.INV_OK
