@@ -457,7 +457,7 @@ def run_ours(args, rank, world, local):
         call()
     torch.cuda.synchronize()
 
-    # ----- the step as a CUDA graph: one decode_layer call (9 kernels) captured
+    # ----- the step as a CUDA graph: one decode_layer call (8 kernels) captured
     # once; every launch argument (buffers, tensor maps) is fixed for the run
     graph = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream()

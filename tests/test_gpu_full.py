@@ -142,7 +142,7 @@ def test_prefill_layer_matches_decode_layer_full_shape(inv):
 def test_prefill_layer_full_shape_oracle_parity(inv):
     """prefill_layer against the float64 oracle layer at the 7B-like shape: a
     700-token prompt in chunks of 300, 77 and 323 rows, so chunk boundaries fall
-    inside 256-key splits and inside the attention's 64-row blocks.  Every row
+    inside 256-key splits and inside the attention's 72-row blocks.  Every row
     of every chunk is within 1e-5 (normwise) of the oracle, and the cache the
     GPU wrote gives decode_layer's bits for the next decoded token."""
     p = host_layer(seed=110)
