@@ -29,6 +29,13 @@
 // For M < 128 only round_up(M, 8) A rows are loaded (the MMA's other rows hold
 // stale data and produce output rows that are never stored).  Persistent grid over tiles ordered
 // N-panel-major so a wave of CTAs shares weight panels and A stays in L2.
+//
+// Two entry points share this body: comp_gemm_kernel (y, optional residual,
+// or the fused SwiGLU epilogue, optionally one side of a producer/consumer
+// pair) and qkv_attn_kernel, the QKV projection whose epilogue applies the
+// rotary embedding and the INT16 KV quantiser to each 128-wide head tile and
+// writes the attention's inputs instead of y (its epilogue warps take column
+// quarters {0, 2} / {1, 3} so that rotate-half partners meet in one thread).
 #include "common.cuh"
 #include "internal.h"
 
