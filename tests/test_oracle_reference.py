@@ -56,6 +56,62 @@ def test_split3_fp16_exact_inputs_equal_fp16_product():
     assert np.array_equal(ref.gemm_fp16_only(A, W), ref.gemm(A, W))
 
 
+def test_fp16_only_rounds_both_operands_to_nearest_even():
+    # Hand-derived binary16 roundings (IEEE 754 round to nearest, ties to even; 10
+    # fraction bits, subnormal step 2^-24) of fp32 inputs that are not binary16:
+    #   1 + 2^-11            tie between 1 and 1 + 2^-10        -> 1           (even)
+    #   1 + 3 2^-11          tie between 1 + 2^-10, 1 + 2^-9    -> 1 + 2^-9    (even)
+    #   1 + 2^-11 + 2^-20    above the tie                      -> 1 + 2^-10
+    #   -(1 + 2^-11 + 2^-20) the same, negated                  -> -(1 + 2^-10)
+    #   2^-25                tie between 0 and 2^-24            -> 0           (even)
+    #   3 2^-26              above half the subnormal step      -> 2^-24
+    #   fp32(0.1)            = 1.6 2^-4; 0.6 * 1024 = 614.4     -> 1638 2^-14
+    #   65519                between 65504 and the overflow tie -> 65504
+    F = Fraction
+    cases = [
+        (F(1) + F(1, 2**11), F(1)),
+        (F(1) + F(3, 2**11), F(1) + F(1, 2**9)),
+        (F(1) + F(1, 2**11) + F(1, 2**20), F(1) + F(1, 2**10)),
+        (-(F(1) + F(1, 2**11) + F(1, 2**20)), -(F(1) + F(1, 2**10))),
+        (F(1, 2**25), F(0)),
+        (F(3, 2**26), F(1, 2**24)),
+        (F(float(np.float32(0.1))), F(1638, 2**14)),
+        (F(65519), F(65504)),
+    ]
+    x = np.array([float(c[0]) for c in cases], np.float32)
+    assert [F(float(v)) for v in x] == [c[0] for c in cases]     # inputs are exact in fp32
+    r = [c[1] for c in cases]
+    n = len(cases)
+    # A row of the cases against a weight whose entries are cases too: a
+    # permutation-like matrix picks each rounded product out, and the last
+    # column sums every rounded A entry times rounded 1 + 3 2^-11.
+    A = x[None, :]
+    W = np.zeros((n, n + 1), np.float32)
+    for i in range(n):
+        W[i, (i + 3) % n] = x[1]
+    W[:, n] = x[1]
+    y = ref.gemm_fp16_only(A, W)
+    for i in range(n):
+        assert F(y[0, (i + 3) % n]) == r[i] * r[1]
+    assert abs(F(y[0, n]) - sum(r) * r[1]) <= F(1, 2**40)
+    # the transposed use: rounded weights against rounded activations
+    yt = ref.gemm_fp16_only(W.T, A.T)
+    for i in range(n):
+        assert F(yt[(i + 3) % n, 0]) == r[i] * r[1]
+
+
+def test_fp16_only_matches_numpy_half_casts():
+    # non-integer data with outliers: numpy's own float16 conversion (an
+    # independent binary16 rounding) on both operands, float64 products
+    A = synth.normal_with_outliers((7, 96), seed=21)
+    W = synth.normal((96, 40), seed=22, std=0.02)
+    want = A.astype(np.float16).astype(np.float64) @ W.astype(np.float16).astype(np.float64)
+    got = ref.gemm_fp16_only(A, W)
+    np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-15)
+    # and the rounding is really there: far from the exact product
+    assert np.abs(got - ref.gemm(A, W)).max() > 1e-5 * np.abs(ref.gemm(A, W)).max()
+
+
 def test_compensated_error_far_below_fp16_only():
     # the GEMM sweep's input model: N(0,1) activations with 0.1% outliers x100,
     # N(0, 0.02) weights
@@ -113,6 +169,75 @@ def test_rope_matches_hf_llama():
     q_hf, _ = apply_rotary_pos_emb(torch.from_numpy(x), torch.from_numpy(x), cos, sin)
     ours = ref.apply_rope(np.transpose(x[0], (1, 0, 2)), pos)           # [t, h, d]
     np.testing.assert_allclose(np.transpose(ours, (1, 0, 2)), q_hf[0].numpy(), rtol=0, atol=1e-13)
+
+
+# ------------------------------------------------------------ KV cache --------
+
+def test_kv_dequant_exact_products_per_row_scale():
+    # codes [H, L, D] with D == L so that a scale broadcast along the wrong axis
+    # still has a valid shape but gives other values
+    H, L = 2, 4
+    codes = np.array([[[32767, -32767, 0, 1],
+                       [-1, 12345, -20000, 7],
+                       [300, -300, 255, -256],
+                       [32767, 32767, -32767, 2]],
+                      [[5, 4, 3, 2],
+                       [-32767, 1, 0, 0],
+                       [11, -13, 17, -19],
+                       [256, 512, -1024, 2048]]], np.int16)
+    scales = np.array([[np.float32(0.1), 0.0, np.float32(2.0**-140), np.float32(3.4e38 / 32767)],
+                       [np.float32(1 / 3), np.float32(2.0**-10), 1.0, np.float32(7.5e-3)]], np.float32)
+    got = enc.kv_dequant(codes, scales)
+    assert got.shape == (H, L, L) and got.dtype == np.float64
+    for h in range(H):
+        for l in range(L):
+            for d in range(L):
+                # a 15-bit integer times a 24-bit significand is exact in float64
+                assert Fraction(got[h, l, d]) == int(codes[h, l, d]) * Fraction(float(scales[h, l]))
+    # a row that is exactly codes x 2^-e quantises to those codes and scale, and
+    # dequantises back to itself
+    k = np.array([32767, -5, 0, 12, -32767, 1024, 3, -2], np.int64)
+    x = np.stack([np.ldexp(k.astype(np.float64), -e) for e in (0, 10, 30)]).astype(np.float32)
+    q, s = enc.kv_quant_int16(x)
+    assert np.array_equal(q, np.broadcast_to(k, q.shape))
+    assert s.tolist() == [1.0, 2.0**-10, 2.0**-30]
+    assert np.array_equal(enc.kv_dequant(q, s), x.astype(np.float64))
+
+
+def test_kv_cache_write_places_codes_and_scales():
+    # rows k * 2^-e with max |k| = 32767 quantise to exactly (k, 2^-e), so the
+    # expected cache contents follow without calling the quantiser
+    S, Hkv, Lmax, D = 3, 2, 6, 8
+    g = np.random.Generator(np.random.PCG64(31))
+    c = ref.KVCache.empty(S, Hkv, Lmax, D)
+    slot = np.array([2, 0, 2, 1])
+    pos = np.array([5, 0, 1, 3])
+    T = len(slot)
+    ints = g.integers(-32766, 32767, size=(T, Hkv, D))
+    ints[:, :, 0] = 32767 * np.where(g.random((T, Hkv)) < 0.5, 1, -1)
+    exps = np.arange(T * Hkv).reshape(T, Hkv) + 3
+    x = np.ldexp(ints.astype(np.float64), -exps[..., None]).astype(np.float32)
+    c.write("k", x, slot, pos)
+    written = set()
+    for t in range(T):
+        for h in range(Hkv):
+            assert np.array_equal(c.k[slot[t], h, pos[t]], ints[t, h])
+            assert c.ks[slot[t], h, pos[t]] == np.float32(2.0**-exps[t, h])
+        written.add((slot[t], pos[t]))
+    # every other position untouched; the value side untouched
+    for s_ in range(S):
+        for p_ in range(Lmax):
+            if (s_, p_) not in written:
+                assert not c.k[s_, :, p_].any() and not c.ks[s_, :, p_].any()
+    assert not c.v.any() and not c.vs.any()
+    # the value side lands in its own arrays; a later write to the same place
+    # replaces the earlier one
+    c.write("v", x[1:2], [2], [5])
+    assert np.array_equal(c.v[2, :, 5], ints[1]) and np.array_equal(c.vs[2, :, 5], c.ks[0, :, 0])
+    c.write("k", x[3:4], [2], [5])
+    assert np.array_equal(c.k[2, :, 5], ints[3])
+    assert np.array_equal(c.ks[2, :, 5], np.float32(2.0**-exps[3]))
+    assert np.array_equal(c.k[2, :, 1], ints[2])
 
 
 # ----------------------------------------------------------- attention --------
