@@ -20,8 +20,9 @@ inputs and D2H of its output inside the timed region), per-kernel times from
 CUDA events recorded around every kernel inside the timed region, the
 roofline of the dominant kernel, SM clocks sampled during the run, and the
 CPU oracle timed on a bounded sample of the same workload.  Components: the
-compensated GEMM at the GEMM-sweep shapes and the decode attention at the
-ragged-length shape, each against its roofline.
+compensated GEMM at the GEMM-sweep shapes, the decode attention at the
+ragged-length shape and RMSNorm at 128 and 8192 rows, each against its
+roofline.
 
 Multi-GPU: replicas only -- every rank runs the full per-GPU workload on its
 own device (weak scaling); the only cross-rank traffic is a barrier and the
@@ -767,6 +768,23 @@ def bench_components(inv, torch, device, peaks, peak_kind):
                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "bytes": byts,
                         "note": "one attn_decode_fixedsplit call (split kernel + ordered combine kernel), "
                                 "L2 flushed between launches"}
+    # RMSNorm at hidden 4096: the decode step's 128 rows and a prompt's 8192
+    # rows, with the layer's binary16 hi/lo output and with fp32 output as well;
+    # bytes = x read + outputs written (gamma is 16 KB and stays in L2)
+    Hn = 4096
+    gamma = torch.from_numpy(synth.uniform((Hn,), seed=50, lo=0.5, hi=1.5)).to(device)
+    norm = {}
+    for rows in (128, 8192):
+        xn = torch.from_numpy(synth.normal((rows, Hn), seed=51)).to(device)
+        for want_y, tag in ((False, "split"), (True, "y_and_split")):
+            t = timed(lambda: inv.rmsnorm_bi(xn, gamma, 1e-6, want_y=want_y, want_split=True))
+            byts = rows * Hn * (4 + 4 + (4 if want_y else 0))
+            gbs = byts / (t * 1e-3) / 1e9
+            norm[f"rows{rows}_{tag}"] = {"us": round(t * 1e3, 2), "bytes": byts, "gbs": round(gbs, 1),
+                                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+        del xn
+    out["rmsnorm"] = {"shapes": norm, "note": "one rmsnorm_bi call (one CTA per row, fixed reduction order), "
+                                              "L2 flushed between launches"}
     assert inv.inv_get_device_status() == inv.INV_OK
     return out
 
@@ -928,6 +946,43 @@ def run_gemm_only(args, local):
                       "steps": args.steps, "warmup": args.warmup}))
 
 
+def run_rmsnorm_only(args, local):
+    """One rmsnorm_bi shape (rows x hidden, binary16 hi/lo output as the layer
+    uses it), timed with CUDA events after a 256 MB write that flushes L2."""
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    from invariant_numerics_b200 import build as _b
+    _b.build()
+    from invariant_numerics_b200 import invnum as inv
+    from invariant_numerics_b200 import synth
+    rows, hidden = args.rmsnorm, args.hidden
+    x = torch.from_numpy(synth.normal((rows, hidden), seed=51)).to(device)
+    gamma = torch.from_numpy(synth.uniform((hidden,), seed=50, lo=0.5, hi=1.5)).to(device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    ts = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        inv.rmsnorm_bi(x, gamma, 1e-6, want_y=False, want_split=True)
+        b.record()
+        b.synchronize()
+        if i >= args.warmup:
+            ts.append(a.elapsed_time(b))
+    st = inv.inv_get_device_status()
+    if st != inv.INV_OK:
+        raise RuntimeError(f"device status {inv.status_string(st)}")
+    peaks, kind = load_peaks()
+    us = statistics.median(ts) * 1e3
+    byts = rows * hidden * 8   # fp32 x read, binary16 hi and lo written
+    gbs = byts / (us * 1e-6) / 1e9
+    print(json.dumps({"metric": "rmsnorm_bi GB/s", "value": round(gbs, 1), "unit": "GB/s",
+                      "config": {"workload": f"rmsnorm_bi rows{rows} hidden{hidden} hi/lo out"}, "us": round(us, 2),
+                      "bytes": byts, "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "peak_source": kind,
+                      "steps": args.steps, "warmup": args.warmup}))
+
+
 def run_prefill_only(args, local):
     """prefill_layer over one T-token sequence (one layer), one shot, timed with
     CUDA events per call; one JSON line (for profiling the prefill kernels)."""
@@ -984,6 +1039,8 @@ def main():
                     help="time one compensated GEMM shape only (one JSON line; for profiling)")
     ap.add_argument("--prefill", type=int, metavar="T",
                     help="time prefill_layer over one T-token sequence only (one JSON line; for profiling)")
+    ap.add_argument("--rmsnorm", type=int, metavar="ROWS",
+                    help="time rmsnorm_bi over ROWS x hidden only (one JSON line; for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -998,6 +1055,8 @@ def main():
         run_gemm_only(args, local)
     elif args.prefill:
         run_prefill_only(args, local)
+    elif args.rmsnorm:
+        run_rmsnorm_only(args, local)
     elif args.impl == "reference":
         run_reference(args, rank, world)
     else:
