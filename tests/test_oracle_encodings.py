@@ -79,6 +79,19 @@ def test_rn16_matches_numpy_cast_on_random_fp32():
     assert ok.all()
 
 
+def test_rn16_matches_numpy_cast_on_every_fp32():
+    """All 2^32 fp32 bit patterns, in blocks of 2^24 over spawned processes."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    from rn16_sweep import check_block
+    block = 1 << 24
+    workers = max(1, min(8, os.cpu_count() or 1))
+    with cf.ProcessPoolExecutor(max_workers=workers, mp_context=mp.get_context("spawn")) as ex:
+        results = list(ex.map(check_block, range(0, 1 << 32, block), [block] * ((1 << 32) // block)))
+    n_bad = sum(r[0] for r in results)
+    assert n_bad == 0, [r[1] for r in results if r[0]][:3]
+
+
 def test_f16_decode_exhaustive_and_roundtrip():
     b = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
     want = b.view(np.float16).astype(np.float64)
