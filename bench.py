@@ -48,6 +48,12 @@ H, HQ, HKV, D, F = 4096, 32, 8, 128, 11008
 BATCH, KV_LEN = 128, 2048
 REFERENCE_SECONDS = 60.0  # timed oracle work of the reference arm, at most
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_FP16_TFLOPS = 2250.0  # dense fp16/bf16 tensor-core figure of the B200 specification (context)
+# Per-launch timings: after the L2 flush the GPU runs a fixed spin of this many
+# clock cycles (~100 us) before the start event, so that the host's enqueue of
+# the timed call (argument checks, tensor maps, launches) overlaps it and the
+# events bracket the call's kernels only.
+HOST_GAP_CYCLES = 200_000
 # DRAM traffic per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)
 # of the step's kernels, recorded by a capture of this benchmark's workload in
 # profiles/dram_traffic.txt together with the SHA-256 of the kernel's source
@@ -688,8 +694,9 @@ def run_ours(args, rank, world, local):
 
 
 def bench_components(inv, torch, device, peaks, peak_kind):
-    """Compensated GEMM (K 4096, N 4096/11008, M 1..1024) and decode attention
-    (32/8 heads, ragged lengths U(128, 8192), B 64), each timed per launch with
+    """Compensated GEMM (K 4096, N 4096/11008, M 1..1024), decode attention
+    (32/8 heads, ragged lengths U(128, 8192), B 64 and its first 1..32 rows)
+    and RMSNorm (hidden 4096, 128 and 8192 rows), each timed per launch with
     CUDA events, L2 flushed between launches."""
     from invariant_numerics_b200 import synth
     out = {}
@@ -700,6 +707,7 @@ def bench_components(inv, torch, device, peaks, peak_kind):
         ts = []
         for r in range(reps + 2):
             flush.zero_()
+            torch.cuda._sleep(HOST_GAP_CYCLES)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             fn()
@@ -726,8 +734,10 @@ def bench_components(inv, torch, device, peaks, peak_kind):
             gbs = byts / (t * 1e-3) / 1e9
             gem[f"M{M}_N{N}"] = {"us": round(t * 1e3, 2), "useful_tflops": round(useful, 2),
                                  "frac_of_peak_over_3": round(useful / (tc_peak / 3), 4),
+                                 "frac_of_nominal_over_3": round(useful / (NOMINAL_FP16_TFLOPS / 3), 4),
                                  "gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
     out["comp_gemm"] = {"shapes": gem, "peak_tflops": tc_peak, "peak_source": f"{peak_kind} bf16_tflops (fp16 = bf16 rate)",
+                        "nominal_tflops": NOMINAL_FP16_TFLOPS,
                         "target": ">= 0.5 x peak / 3 useful at M 256, 1024"}
 
     B = 64
@@ -747,9 +757,21 @@ def bench_components(inv, torch, device, peaks, peak_kind):
     o = torch.empty_like(q)
     ws = torch.empty(inv.attn_decode_workspace_size(B, HQ, 8192), dtype=torch.uint8, device=device)
     t = timed(lambda: inv.attn_decode_fixedsplit(q, cache, slot, lens_d, 0.08838834764831845, out=o, workspace=ws))
-    S = (lens.astype(np.int64) + 255) // 256
-    byts = int(lens.astype(np.int64).sum()) * HKV * 520 + B * HQ * D * 4 * 2 + int(S.sum()) * HQ * (D + 2) * 4 * 2
+    def attn_bytes(ls):
+        S = (ls.astype(np.int64) + 255) // 256
+        return int(ls.astype(np.int64).sum()) * HKV * 520 + len(ls) * HQ * D * 4 * 2 + int(S.sum()) * HQ * (D + 2) * 4 * 2
+    byts = attn_bytes(lens)
     gbs = byts / (t * 1e-3) / 1e9
+    # the same call on the first Bs sequences of the cache
+    sweep = {}
+    for Bs in (1, 2, 4, 8, 16, 32, 64):
+        qs, ss, ls, os_ = q[:Bs].contiguous(), slot[:Bs].contiguous(), lens_d[:Bs].contiguous(), o[:Bs]
+        ts = timed(lambda: inv.attn_decode_fixedsplit(qs, cache, ss, ls, 0.08838834764831845, out=os_, workspace=ws))
+        bs = attn_bytes(lens[:Bs])
+        sweep[f"B{Bs}"] = {"mean_len": float(lens[:Bs].mean()), "us": round(ts * 1e3, 2), "bytes": bs,
+                           "gbs": round(bs / (ts * 1e-3) / 1e9, 1),
+                           "frac_hbm": round(bs / (ts * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    out["attention_batch_sweep"] = sweep
     # LAMP variant on the same workload: time, recompute rate, distance from the plain call
     lamp = {}
     for tau in (0.01, 0.1, 1.0):
@@ -927,6 +949,7 @@ def run_gemm_only(args, local):
     ts = []
     for i in range(args.warmup + args.steps):
         flush.zero_()
+        torch.cuda._sleep(HOST_GAP_CYCLES)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         inv.comp_gemm(hi, lo, P, e, out=y)
@@ -963,6 +986,7 @@ def run_rmsnorm_only(args, local):
     ts = []
     for i in range(args.warmup + args.steps):
         flush.zero_()
+        torch.cuda._sleep(HOST_GAP_CYCLES)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         inv.rmsnorm_bi(x, gamma, 1e-6, want_y=False, want_split=True)

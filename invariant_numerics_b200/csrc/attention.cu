@@ -517,6 +517,7 @@ __global__ void __launch_bounds__(THREADS, 3)
                       int n_slots, int max_len, int len_limit, int S_max, float sigma, float* __restrict__ part_o,
                       float2* __restrict__ part_ml, int* status, long long wait_ns, float tau, uint8_t* sel,
                       int64_t sel_ld) {
+  inv::grid_launch_dependents();  // the combine kernel may be scheduled once every CTA has started
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int G = Hq / Hkv;
   const int L = len[b], sl = slot[b];
@@ -633,6 +634,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                               const float* __restrict__ vscale, int sl, int p0, int T, int Hq, int Hkv, int max_len,
                               int S_max, float sigma, float* __restrict__ part_o, float2* __restrict__ part_ml,
                               int* status, long long wait_ns, int n_slots) {
+  inv::grid_launch_dependents();  // the combine kernel may be scheduled once every CTA has started
   const int s = blockIdx.x, h = blockIdx.y, rb = blockIdx.z;
   const int G = Hq / Hkv;
   const int key0 = s * SPLIT;
@@ -708,11 +710,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   if (tid == 0) inv::mbar_wait(&sm.bar_kv, 0, wait_ns, nullptr, status);
 }
 
-// One warp per (row, head): fold splits s = 0, 1, ... in order.
+// One warp per (row, head): fold splits s = 0, 1, ... in order.  Launched as a
+// programmatic dependent of the split kernel: it waits for that grid's
+// completion before its first load.
 __global__ void attn_combine_kernel(const float* __restrict__ part_o, const float2* __restrict__ part_ml,
                                     const int32_t* __restrict__ len, int B, int Hq, int S_max, int len_limit,
                                     float* __restrict__ out, __half* __restrict__ out_hi, __half* __restrict__ out_lo,
                                     int* status) {
+  inv::grid_wait_prerequisites();
   const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (wid >= (int64_t)B * Hq) return;
@@ -724,58 +729,43 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o, const floa
   const int b = (int)(wid / Hq);
   const float2* ml = part_ml + wid * S_max;
   const float4* po = reinterpret_cast<const float4*>(part_o + wid * S_max * 128) + lane;
-  // The first 8 splits' (m, l) and o are requested together with len[b]: one
-  // memory round trip for KV lengths up to 2048.  Entries past the row's own
-  // split count are loaded (inside the partials buffer) but never used.
+  // One memory round trip for len[b], the (m, l) of the first 32 splits (lane
+  // j holds split j) and this lane's o of the first PF splits; entries past
+  // the row's own split count are loaded (inside the partials buffer) but
+  // never used.
   constexpr int PF = 8;
-  float2 v0[PF];
-  float4 o0[PF];
+  const float2 ml0 = lane < S_max ? ml[lane] : make_float2(-INFINITY, 0.0f);
+  float4 o[PF];
 #pragma unroll
-  for (int j = 0; j < PF; ++j) {
-    v0[j] = j < S_max ? ml[j] : make_float2(-INFINITY, 0.0f);
-    o0[j] = j < S_max ? po[j * 32] : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
+  for (int j = 0; j < PF; ++j) o[j] = j < S_max ? po[j * 32] : make_float4(0.f, 0.f, 0.f, 0.f);
   const int L = len[b];
   float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
   if (L >= 1 && L <= len_limit) {
     const int S = (L + SPLIT - 1) / SPLIT;
-    float M = -INFINITY;  // exact max: order does not matter
+    float M = lane < S ? ml0.x : -INFINITY;  // exact max: order does not matter
+    for (int c = 32; c < S; c += 32) M = fmaxf(M, lane + c < S ? ml[lane + c].x : -INFINITY);
 #pragma unroll
-    for (int j = 0; j < PF; ++j)
-      if (j < S) M = fmaxf(M, v0[j].x);
-    for (int s0 = PF; s0 < S; s0 += 8) {
-      float2 v[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = s0 + j < S ? ml[s0 + j] : make_float2(-INFINITY, 0.0f);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) M = fmaxf(M, v[j].x);
-    }
+    for (int k = 16; k >= 1; k >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, k));
     float l = 0.0f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    // splits folded in ascending order
+    float fc = 0.0f, lc = 0.0f;  // this lane's split of the current 32: exp(m - M) and l
+    // splits folded in ascending order; split s's factor and l come from lane s % 32
+    for (int s0 = 0; s0 < S; s0 += PF) {
+      if ((s0 & 31) == 0) {
+        const float2 mlc = s0 == 0 ? ml0 : (lane + s0 < S ? ml[lane + s0] : make_float2(-INFINITY, 0.0f));
+        fc = lane + s0 < S ? expf(__fsub_rn(mlc.x, M)) : 0.0f;
+        lc = mlc.y;
+      }
+      if (s0 > 0) {  // PF loads in flight
 #pragma unroll
-    for (int j = 0; j < PF; ++j) {
-      if (j >= S) break;
-      const float f = expf(__fsub_rn(v0[j].x, M));
-      l = __fadd_rn(l, __fmul_rn(v0[j].y, f));
-      acc.x = __fadd_rn(acc.x, __fmul_rn(o0[j].x, f));
-      acc.y = __fadd_rn(acc.y, __fmul_rn(o0[j].y, f));
-      acc.z = __fadd_rn(acc.z, __fmul_rn(o0[j].z, f));
-      acc.w = __fadd_rn(acc.w, __fmul_rn(o0[j].w, f));
-    }
-    for (int s0 = PF; s0 < S; s0 += 8) {  // 8 loads in flight
-      float2 v[8];
-      float4 o[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        v[j] = s0 + j < S ? ml[s0 + j] : make_float2(-INFINITY, 0.0f);
-        o[j] = s0 + j < S ? po[(s0 + j) * 32] : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < PF; ++j) o[j] = s0 + j < S ? po[(s0 + j) * 32] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < PF; ++j) {
         if (s0 + j >= S) break;
-        const float f = expf(__fsub_rn(v[j].x, M));
-        l = __fadd_rn(l, __fmul_rn(v[j].y, f));
+        const float f = __shfl_sync(0xffffffffu, fc, (s0 + j) & 31);
+        const float lj = __shfl_sync(0xffffffffu, lc, (s0 + j) & 31);
+        l = __fadd_rn(l, __fmul_rn(lj, f));
         acc.x = __fadd_rn(acc.x, __fmul_rn(o[j].x, f));
         acc.y = __fadd_rn(acc.y, __fmul_rn(o[j].y, f));
         acc.z = __fadd_rn(acc.z, __fmul_rn(o[j].z, f));
@@ -818,6 +808,30 @@ size_t attn_workspace_bytes(int B, int Hq, int max_len_bound) {
 }
 
 // The decode split kernel (plain or LAMP), then the ordered combine.
+// The ordered combine, one warp per (row, head), launched as a programmatic
+// dependent of the split kernel just enqueued on the stream (its launch
+// overlaps that grid's last wave; it waits for the grid before reading).
+static int launch_combine(const float* part_o, const float2* part_ml, const int32_t* len, int rows, int Hq, int S_max,
+                          int len_limit, float* out, uint16_t* out_hi, uint16_t* out_lo, cudaStream_t s) {
+  const int64_t warps = (int64_t)rows * Hq;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)((warps * 32 + 255) / 256));
+  lc.blockDim = dim3(256);
+  lc.dynamicSmemBytes = 0;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&lc, attn_combine_kernel, part_o, part_ml, len, rows, Hq, S_max, len_limit,
+                                           out, reinterpret_cast<__half*>(out_hi), reinterpret_cast<__half*>(out_lo),
+                                           status_ptr());
+  if (e != cudaSuccess) return INV_ERR_CUDA;
+  INV_CHECK_LAUNCH();
+  return INV_OK;
+}
+
 template <bool kLamp>
 static int launch_decode(const float* q, int B, int Hq, const inv_kv_cache& c, const int32_t* slot,
                          const int32_t* len, int max_len_bound, float sigma, float* out, uint16_t* out_hi,
@@ -850,12 +864,9 @@ static int launch_decode(const float* q, int B, int Hq, const inv_kv_cache& c, c
       part_o, part_ml, status_ptr(), wait_limit_ns(), tau, sel, sel_ld);
   INV_CHECK_LAUNCH();
   trace_record(2 * trace_base + 1, s);
-  const int64_t warps = (int64_t)B * Hq;
   trace_record(2 * trace_base + 2, s);
-  attn_combine_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(
-      part_o, part_ml, len, B, Hq, S_max, max_len_bound, out, reinterpret_cast<__half*>(out_hi),
-      reinterpret_cast<__half*>(out_lo), status_ptr());
-  INV_CHECK_LAUNCH();
+  rc = launch_combine(part_o, part_ml, len, B, Hq, S_max, max_len_bound, out, out_hi, out_lo, s);
+  if (rc != INV_OK) return rc;
   trace_record(2 * trace_base + 3, s);
   return INV_OK;
 }
@@ -896,12 +907,9 @@ int launch_attention_prefill(const float* q, int T, int Hq, const inv_kv_cache& 
                                                                 part_ml, status_ptr(), wait_limit_ns(), c.n_slots);
   INV_CHECK_LAUNCH();
   trace_record(2 * trace_base + 1, s);
-  const int64_t warps = (int64_t)T * Hq;
   trace_record(2 * trace_base + 2, s);
-  attn_combine_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(
-      part_o, part_ml, len, T, Hq, S_max, max_len_bound, out, reinterpret_cast<__half*>(out_hi),
-      reinterpret_cast<__half*>(out_lo), status_ptr());
-  INV_CHECK_LAUNCH();
+  const int rcc = launch_combine(part_o, part_ml, len, T, Hq, S_max, max_len_bound, out, out_hi, out_lo, s);
+  if (rcc != INV_OK) return rcc;
   trace_record(2 * trace_base + 3, s);
   return INV_OK;
 }
