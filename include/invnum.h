@@ -241,7 +241,8 @@ INV_API int kv_quant_int16(const float* x, int T, int64_t ld_x, const int32_t* s
  * dual-FP16 unpacked codes (code = 256 h + l, both exact in binary16) and the
  * hi/lo split of q, its own max, exp-sum and value sum; the splits are then
  * folded in ascending s.  Nothing depends on other rows or on len beyond the
- * row's own split count.
+ * row's own split count.  Two kernels on `stream`: the split kernel, then the
+ * ordered combine as its programmatic dependent.
  *   q        : fp32 [B][n_heads][128], 16-byte aligned.
  *   len      : int32 [B], 1 <= len[b] <= cache->max_len.
  *   max_len_bound : host upper bound on every len[b] (<= 0: cache->max_len);
@@ -365,12 +366,12 @@ INV_API int rmsnorm_bi(const float* x, const float* gamma, int64_t rows, int hid
  *                 returns 0 for L <= 0).  Calls that overlap on the GPU need
  *                 separate workspaces.
  * Stream work: the layer's kernels only, all on `stream` (the QKV GEMM also
- * clears the workspace's gate/up tile counters).  The W_down GEMM
- * is launched as a
- * programmatic dependent of the gate/up GEMM and starts during its last
+ * clears the workspace's gate/up tile counters).  The W_down GEMM is launched
+ * as a programmatic dependent of the gate/up GEMM and starts during its last
  * partial wave, loading each K block of a once the gate/up tile that stores it
- * has published it (no change to any product or sum).  All of this may be
- * captured into a CUDA graph.
+ * has published it (no change to any product or sum).  The attention combine
+ * is a programmatic dependent of the split kernel and waits for that grid
+ * before its first load.  All of this may be captured into a CUDA graph.
  * Errors: as the component calls; INV_ERR_WORKSPACE.
  * ------------------------------------------------------------------------ */
 typedef struct {
