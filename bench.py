@@ -63,17 +63,18 @@ KERNEL_SOURCES = {"comp_gemm_kernel": "comp_gemm.cu", "qkv_attn_kernel": "comp_g
                   "attn_split_kernel": "attention.cu"}
 
 
-def captured_traffic(kernel: str, workload: str):
+def captured_traffic(kernel: str, workload: str, record: str = TRAFFIC_RECORD,
+                     src_dir: str = os.path.join(ROOT, "invariant_numerics_b200", "csrc")):
     """(bytes per launch, note) from the capture record, or (None, why)."""
     import hashlib
     try:
-        with open(TRAFFIC_RECORD) as f:
+        with open(record) as f:
             rec = json.load(f).get(kernel)
     except Exception:
         return None, "no capture record"
     if not rec or rec.get("workload") != workload:
         return None, "no capture of this workload"
-    src = os.path.join(ROOT, "invariant_numerics_b200", "csrc", KERNEL_SOURCES[kernel])
+    src = os.path.join(src_dir, KERNEL_SOURCES[kernel])
     with open(src, "rb") as f:
         sha = hashlib.sha256(f.read()).hexdigest()
     if sha != rec.get("source_sha256"):
@@ -89,13 +90,12 @@ def _numeric_leaves(obj, path=()):
         yield "/".join(path), float(obj)
 
 
-def load_peaks():
+def load_peaks(path: str = os.path.join(ROOT, "MEASURED_PEAKS.json")):
     """Measured peaks of this GPU model (HBM copy GB/s, dense bf16 TFLOP/s as
     a burst and sustained), read from MEASURED_PEAKS.json at the repository
     root whatever its nesting: each figure is the first numeric entry whose
     key path names it.  A figure the file lacks (or a missing file) takes the
     fallback value, and the returned kind says which."""
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             leaves = list(_numeric_leaves(json.load(f)))
