@@ -10,15 +10,16 @@
 // exact binary16 numbers, so two 16-bit tensor-core products recover q/256
 // exactly before fp32 accumulation.
 //
-// Split kernel: one CTA (4 warps) per (row b, kv head, split s).  The 256 x 128
-// K codes arrive by TMA (2-D, 128-byte swizzle) into 64 KB of shared memory;
-// every warp owns 64 keys.  Scores S^T = K Q^T use mma.m16n8k16 with the 16
-// keys of an m-tile as rows and the 8 columns [q_hi, q_lo] x 4 query heads of
-// the GQA group (q split like heal_split) as N.  The split max, exp, sum and
-// a per-(split, head) power-of-two scaling of w = p s_V follow; the V codes
-// then overwrite the K buffer and O^T = V^T W runs with d as rows and
-// [w_hi, w_lo] x 4 heads as columns.  Warps' partial sums are added in warp
-// order.  Output per (row, head, split): (m, l, o[128]).
+// Split kernel: one CTA (4 warps) per (row b, kv head, split s); every warp
+// owns 64 keys and stages them by TMA (2-D, 128-byte swizzle) as two halves of
+// 32 keys in its own 8 KB slot, so a CTA needs ~40 KB of shared memory and 5
+// CTAs share an SM.  Scores S^T = K Q^T use mma.m16n8k16 with the 16 keys of
+// an m-tile as rows and the 8 columns [q_hi, q_lo] x 4 query heads of the GQA
+// group (q split like heal_split) as N.  The split max, exp, sum and a
+// per-(split, head) power-of-two scaling of w = p s_V follow; the V halves
+// then take the K slots and O^T = V^T W runs with d as rows and [w_hi, w_lo] x
+// 4 heads as columns.  Warps' partial sums are added in warp order.  Output per
+// (row, head, split): (m, l, o[128]).
 // Combine kernel: one warp per (row, head) folds the splits s = 0, 1, ... in
 // order, o / l, and writes fp32 plus the binary16 hi/lo split.
 //
@@ -53,17 +54,25 @@ struct LampArgs {
   int64_t sel_head_stride;
 };
 
+// The decode kernel stages each warp's 64 keys as two halves of 32 keys in one
+// 8 KB slot (K first half, second half, then V likewise), so that a CTA needs
+// ~39 KB of shared memory and 5 CTAs fit on an SM.
+constexpr int HALF_KEYS = 32;
+constexpr int HBOX_BYTES = HALF_KEYS * 64 * 2;  // 32 keys x 64 d x int16
+constexpr int WARP_SLOT = 2 * HBOX_BYTES;       // 32 keys x 128 d
+
 struct __align__(1024) DecodeSmem {
-  uint8_t codes[CODE_BYTES];   // K codes, then V codes, then the warp exchange of O
-  float qs[4 * 128];           // q of the row's G query heads (bulk copy with K)
-  uint32_t qfrag[512];         // their hi/lo MMA fragments
+  uint8_t codes[4 * WARP_SLOT];  // per warp: K halves, then V halves; then the warp exchange of O
+  float qs[4 * 128];             // q of the row's G query heads (bulk copy with K)
+  uint32_t qfrag[512];           // their hi/lo MMA fragments
   float ks[SPLIT];
   float vs[SPLIT];
   RowScratch rs;
-  uint64_t bar_k, bar_q, bar_v[4];  // V: one barrier per warp (its 64 keys)
+  uint64_t bar_k, bar_q, bar_k2[4], bar_v[4], bar_v2[4];  // K first halves (all warps); per warp the rest
   int abort;
 };
 constexpr size_t kDecodeSmem = sizeof(DecodeSmem) + 1024;
+static_assert(4 * 4 * 128 * sizeof(float) <= sizeof(DecodeSmem::codes), "the O exchange aliases the codes");
 
 // Prefill: PF_GROUPS groups of 128 threads each run the per-row code on PF_R
 // rows at a time of the block (every unpacked K/V fragment feeds PF_R rows'
@@ -129,6 +138,22 @@ __device__ __forceinline__ uint32_t code_addr(uint32_t base, int kk, int d0) {
          ((((d0 & 63) >> 3) ^ (r & 7)) << 4);
 }
 
+// The same for the decode kernel's half staging: warp slot kk/64, d half d0/64
+// (a 32-row box), row kk%32, 16-byte chunk ((d0%64)/8) xor (row%8); each
+// warp's two 32-key halves share its slot one after the other.
+__device__ __forceinline__ uint32_t code_addr_half(uint32_t base, int kk, int d0) {
+  const int r = kk & 31;
+  return base + (kk >> 6) * WARP_SLOT + (d0 >> 6) * HBOX_BYTES + r * 128 + ((((d0 & 63) >> 3) ^ (r & 7)) << 4);
+}
+
+template <bool kHalf>
+__device__ __forceinline__ uint32_t caddr(uint32_t base, int kk, int d0) {
+  if constexpr (kHalf)
+    return code_addr_half(base, kk, d0);
+  else
+    return code_addr(base, kk, d0);
+}
+
 __device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
   return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
 }
@@ -162,7 +187,7 @@ struct RowSet {
 //   issue_v / wait_v : hooks around the first V access.  issue_v runs in every
 //          thread once its warp has finished reading K (a warp reads and later
 //          overwrites only the codes of its own 64 keys); the decode kernel
-//          loads that warp's V codes into the warp's K slot there.
+//          loads the first half of that warp's V codes into its slot there.
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
@@ -206,13 +231,18 @@ __device__ __forceinline__ void write_q_fragments(int tid, const RowSet<R>& rows
 // scores whose relaxed criterion 2 exp(y_lo - m_lo) |y_lo| exceeds tau (m_lo
 // the split's largest finite low-precision score; non-finite ones always)
 // keep the full-precision value; the others continue with y_lo.
-template <int R, bool kReuse, bool kLamp, bool kQReady, class Sync, class IssueV, class WaitV>
+// kHalf: the codes are staged in 32-key halves (code_addr_half); mid_k and
+// mid_v run in every thread of a warp before its third m-tile of the scores
+// and of P.V, once the warp has read its first half: they bring the second
+// half of the warp's K or V codes into its slot and return the warp's ok.
+template <int R, bool kReuse, bool kLamp, bool kQReady, bool kHalf, class Sync, class IssueV, class WaitV, class MidK,
+          class MidV>
 __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& rows, int G, uint32_t kbase,
                                            uint32_t vbase, const float* ks, const float* vs, RowScratch* rs,
                                            float* xo, uint32_t* qfrag, float sigma, int64_t head_stride_o,
                                            int64_t head_stride_ml,
                                            bool ok, int* status, const LampArgs& lamp, IssueV issue_v,
-                                           WaitV wait_v) {
+                                           WaitV wait_v, MidK mid_k, MidV mid_v) {
   static_assert(!kLamp || R == 1, "the low-precision pass is per row");
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
   int n_max = 0;
@@ -248,6 +278,9 @@ __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& 
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt) {
     const int kb = warp * 64 + mt * 16;
+    if constexpr (kHalf) {
+      if (mt == 2) ok = mid_k(ok);
+    }
 #pragma unroll
     for (int r = 0; r < R; ++r) tsc[r][mt][0] = tsc[r][mt][1] = -INFINITY;
     if constexpr (kLamp) tlo[mt][0] = tlo[mt][1] = -INFINITY;
@@ -258,8 +291,8 @@ __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& 
         const float* qh = lamp.q + c * 128;
 #pragma unroll 2
         for (int d0 = 0; d0 < 128; d0 += 8) {
-          const uint4 c1 = lds128(code_addr(kbase, kb + g, d0));
-          const uint4 c2 = lds128(code_addr(kbase, kb + g + 8, d0));
+          const uint4 c1 = lds128(caddr<kHalf>(kbase, kb + g, d0));
+          const uint4 c2 = lds128(caddr<kHalf>(kbase, kb + g + 8, d0));
           const uint32_t w1[4] = {c1.x, c1.y, c1.z, c1.w}, w2[4] = {c2.x, c2.y, c2.z, c2.w};
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -292,7 +325,7 @@ __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& 
 #pragma unroll
       for (int ks_ = 0; ks_ < 8; ++ks_) {
         uint32_t a[4], ah[4], al[4];
-        ldsm_x4(code_addr(kbase, lkey, 16 * ks_ + (lane >> 4) * 8), a);
+        ldsm_x4(caddr<kHalf>(kbase, lkey, 16 * ks_ + (lane >> 4) * 8), a);
 #pragma unroll
         for (int i = 0; i < 4; ++i) unpack_dual(a[i], ah[i], al[i]);
 #pragma unroll
@@ -427,6 +460,9 @@ __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& 
 #pragma unroll
   for (int mt = 0; mt < 4; ++mt) {
     const int kb = warp * 64 + mt * 16;
+    if constexpr (kHalf) {
+      if (mt == 2) ok = mid_v(ok);
+    }
     // B fragment of O^T = V^T W: rows k = keys, column g = head g/2 (hi/lo)
     uint32_t b0[R], b1[R];
 #pragma unroll
@@ -444,7 +480,7 @@ __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& 
 #pragma unroll
       for (int dt = 0; dt < 8; ++dt) {
         uint32_t a[4], ah[4], al[4];
-        ldsm_x4_t(code_addr(vbase, lkey, 16 * dt + ((lane >> 3) & 1) * 8), a);
+        ldsm_x4_t(caddr<kHalf>(vbase, lkey, 16 * dt + ((lane >> 3) & 1) * 8), a);
 #pragma unroll
         for (int i = 0; i < 4; ++i) unpack_dual(a[i], ah[i], al[i]);
 #pragma unroll
@@ -510,7 +546,7 @@ __device__ __forceinline__ void split_rows(int tid, Sync sync, const RowSet<R>& 
 // Decode: one CTA per (row b, kv head h, split s).  kLamp: the LAMP variant
 // (tau, and the recompute flags sel [B][Hq][sel_ld] or null).
 template <bool kLamp>
-__global__ void __launch_bounds__(THREADS, 3)
+__global__ void __launch_bounds__(THREADS, 5)
     attn_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const float* __restrict__ q, const float* __restrict__ kscale, const float* __restrict__ vscale,
                       const int32_t* __restrict__ slot, const int32_t* __restrict__ len, int Hq, int Hkv,
@@ -553,19 +589,25 @@ __global__ void __launch_bounds__(THREADS, 3)
   if (tid == 0) {
     inv::mbar_init(&sm.bar_k, 1);
     inv::mbar_init(&sm.bar_q, 1);
-    for (int w = 0; w < 4; ++w) inv::mbar_init(&sm.bar_v[w], 1);
+    for (int w = 0; w < 4; ++w) {
+      inv::mbar_init(&sm.bar_k2[w], 1);
+      inv::mbar_init(&sm.bar_v[w], 1);
+      inv::mbar_init(&sm.bar_v2[w], 1);
+    }
     sm.abort = 0;
     inv::fence_mbar_init();
   }
   __syncthreads();
+  // warp w holds keys 64 w .. 64 w + 63 of the split: its first half exists
+  // when 64 w < n (w < nbox), its second half when 64 w + 32 < n
   if (tid == 0) {
     // q on its own barrier: its fragments are split while the codes land
     inv::mbar_arrive_expect_tx(&sm.bar_q, G * 128 * 4);
     inv::bulk_load(sm.qs, q + obase * 128, (uint32_t)(G * 128 * 4), &sm.bar_q);
-    inv::mbar_arrive_expect_tx(&sm.bar_k, nbox * 2 * BOX_BYTES);
-    for (int bx = 0; bx < nbox; ++bx) {
-      inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES, &tm_k, &sm.bar_k, 0, row0 + 64 * bx);
-      inv::tma_load_2d(sm.codes + bx * 2 * BOX_BYTES + BOX_BYTES, &tm_k, &sm.bar_k, 64, row0 + 64 * bx);
+    inv::mbar_arrive_expect_tx(&sm.bar_k, nbox * WARP_SLOT);
+    for (int w = 0; w < nbox; ++w) {
+      inv::tma_load_2d(sm.codes + w * WARP_SLOT, &tm_k, &sm.bar_k, 0, row0 + 64 * w);
+      inv::tma_load_2d(sm.codes + w * WARP_SLOT + HBOX_BYTES, &tm_k, &sm.bar_k, 64, row0 + 64 * w);
     }
   }
   // the scales go to registers first (stored after the q fragments are done)
@@ -592,24 +634,43 @@ __global__ void __launch_bounds__(THREADS, 3)
   if (lane == 0 && ok) ok = inv::mbar_wait(&sm.bar_k, 0, wait_ns, &sm.abort, status);
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 
-  bool v_issued = false;
+  const int warp = tid >> 5;
+  const bool has_first = warp < nbox, has_second = 64 * warp + HALF_KEYS < n;
+  uint8_t* slot_ptr = sm.codes + warp * WARP_SLOT;
+  // one bounded load of 32 keys x 128 d into this warp's slot, after every
+  // lane's reads of the slot (generic proxy) are ordered before the copy
+  bool issued_k2 = false, issued_v = false, issued_v2 = false;
+  const auto reload = [&](bool okr, const CUtensorMap* tm, uint64_t* bar, int key_row, bool& issued) {
+    inv::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && okr) {
+      issued = true;
+      inv::mbar_arrive_expect_tx(bar, WARP_SLOT);
+      inv::tma_load_2d(slot_ptr, tm, bar, 0, key_row);
+      inv::tma_load_2d(slot_ptr + HBOX_BYTES, tm, bar, 64, key_row);
+    }
+  };
+  const auto await = [&](bool okw, uint64_t* bar) {
+    if (lane == 0 && okw) okw = inv::mbar_wait(bar, 0, wait_ns, &sm.abort, status);
+    return __shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0;
+  };
   const LampArgs lamp = {tau, sm.qs, sel != nullptr ? sel + obase * sel_ld + key0 : nullptr, sel_ld};
-  split_rows<1, false, kLamp, true>(
+  split_rows<1, false, kLamp, true, true>(
       tid, []() { __syncthreads(); }, rows, G, cbase, cbase, sm.ks, sm.vs, &sm.rs,
       reinterpret_cast<float*>(sm.codes), sm.qfrag, sigma, (int64_t)S_max * 128, (int64_t)S_max, ok, status, lamp,
-      [&]() {  // this warp is done with its K codes: bring its V codes into the same slot
-        const int warp = tid >> 5;
-        if (lane == 0 && ok && warp < nbox) {
-          v_issued = true;
-          inv::mbar_arrive_expect_tx(&sm.bar_v[warp], 2 * BOX_BYTES);
-          inv::tma_load_2d(sm.codes + warp * 2 * BOX_BYTES, &tm_v, &sm.bar_v[warp], 0, row0 + 64 * warp);
-          inv::tma_load_2d(sm.codes + warp * 2 * BOX_BYTES + BOX_BYTES, &tm_v, &sm.bar_v[warp], 64, row0 + 64 * warp);
-        }
+      [&]() {  // this warp is done with its K codes: bring its first V half into the same slot
+        if (has_first) reload(ok, &tm_v, &sm.bar_v[warp], row0 + 64 * warp, issued_v);
       },
-      [&](bool okv) {
-        const int warp = tid >> 5;
-        if (lane == 0 && okv && warp < nbox) okv = inv::mbar_wait(&sm.bar_v[warp], 0, wait_ns, &sm.abort, status);
-        return __shfl_sync(0xffffffffu, okv ? 1 : 0, 0) != 0;
+      [&](bool okv) { return has_first ? await(okv, &sm.bar_v[warp]) : okv; },
+      [&](bool okk) {  // scores of the first K half done: the second K half
+        if (!has_second) return okk;
+        reload(okk, &tm_k, &sm.bar_k2[warp], row0 + 64 * warp + HALF_KEYS, issued_k2);
+        return await(okk, &sm.bar_k2[warp]);
+      },
+      [&](bool okv) {  // P.V of the first V half done: the second V half
+        if (!has_second) return okv;
+        reload(okv, &tm_v, &sm.bar_v2[warp], row0 + 64 * warp + HALF_KEYS, issued_v2);
+        return await(okv, &sm.bar_v2[warp]);
       });
   // No copy may still be landing in this CTA's shared memory when it exits
   // (only possible after a timed-out wait; immediate otherwise).
@@ -617,7 +678,11 @@ __global__ void __launch_bounds__(THREADS, 3)
     inv::mbar_wait(&sm.bar_q, 0, wait_ns, nullptr, status);
     inv::mbar_wait(&sm.bar_k, 0, wait_ns, nullptr, status);
   }
-  if (lane == 0 && v_issued) inv::mbar_wait(&sm.bar_v[tid >> 5], 0, wait_ns, nullptr, status);
+  if (lane == 0) {
+    if (issued_k2) inv::mbar_wait(&sm.bar_k2[warp], 0, wait_ns, nullptr, status);
+    if (issued_v) inv::mbar_wait(&sm.bar_v[warp], 0, wait_ns, nullptr, status);
+    if (issued_v2) inv::mbar_wait(&sm.bar_v2[warp], 0, wait_ns, nullptr, status);
+  }
 }
 
 // Prefill: rows r = 0..T-1 of one sequence (slot sl) at positions p0 + r.
@@ -702,9 +767,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     }
     // the q fragments of the rows use the start of the group's exchange buffer,
     // which is written only after the last V read
-    split_rows<PF_R, true, false, false>(gtid, group_sync, rows, G, kbase, vbase, sm.ks, sm.vs, sm.rs[grp], sm.xo[grp][0],
-                                  reinterpret_cast<uint32_t*>(sm.xo[grp][0]),
+    split_rows<PF_R, true, false, false, false>(gtid, group_sync, rows, G, kbase, vbase, sm.ks, sm.vs, sm.rs[grp],
+                                  sm.xo[grp][0], reinterpret_cast<uint32_t*>(sm.xo[grp][0]),
                                   sigma, (int64_t)S_max * 128, (int64_t)S_max, ok, status, LampArgs{}, []() {},
+                                  [](bool okv) { return okv; }, [](bool okk) { return okk; },
                                   [](bool okv) { return okv; });
   }
   if (tid == 0) inv::mbar_wait(&sm.bar_kv, 0, wait_ns, nullptr, status);
@@ -843,17 +909,20 @@ static int launch_decode(const float* q, int B, int Hq, const inv_kv_cache& c, c
   float* part_o = static_cast<float*>(ws);
   float2* part_ml = reinterpret_cast<float2*>(part_o + (size_t)B * Hq * S_max * 128);
   const uint64_t rows = (uint64_t)c.n_slots * c.n_kv_heads * c.max_len;
-  CUtensorMap tk, tv;
-  int rc = make_tensor_map_2d(&tk, c.k, CU_TENSOR_MAP_DATA_TYPE_UINT16, 128, rows, 256, 64, 64,
+  CUtensorMap tk, tv;  // boxes of 32 keys x 64 d (each warp stages its keys in two halves)
+  int rc = make_tensor_map_2d(&tk, c.k, CU_TENSOR_MAP_DATA_TYPE_UINT16, 128, rows, 256, 64, HALF_KEYS,
                               CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != INV_OK) return rc;
-  rc = make_tensor_map_2d(&tv, c.v, CU_TENSOR_MAP_DATA_TYPE_UINT16, 128, rows, 256, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  rc = make_tensor_map_2d(&tv, c.v, CU_TENSOR_MAP_DATA_TYPE_UINT16, 128, rows, 256, 64, HALF_KEYS,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != INV_OK) return rc;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     if (cudaFuncSetAttribute(attn_split_kernel<kLamp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kDecodeSmem) != cudaSuccess)
+                             (int)kDecodeSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_split_kernel<kLamp>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return INV_ERR_CUDA;
     attr_set[dev] = true;
   }
