@@ -54,6 +54,14 @@ NOMINAL_FP16_TFLOPS = 2250.0  # dense fp16/bf16 tensor-core figure of the B200 s
 # the timed call (argument checks, tensor maps, launches) overlaps it and the
 # events bracket the call's kernels only.
 HOST_GAP_CYCLES = 200_000
+
+
+def host_gap(torch) -> None:
+    """The fixed GPU spin before a per-launch start event (skipped if this
+    PyTorch build has no spin kernel)."""
+    spin = getattr(torch.cuda, "_sleep", None)
+    if spin is not None:
+        spin(HOST_GAP_CYCLES)
 # DRAM traffic per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)
 # of the step's kernels, recorded by a capture of this benchmark's workload in
 # profiles/dram_traffic.txt together with the SHA-256 of the kernel's source
@@ -707,7 +715,7 @@ def bench_components(inv, torch, device, peaks, peak_kind):
         ts = []
         for r in range(reps + 2):
             flush.zero_()
-            torch.cuda._sleep(HOST_GAP_CYCLES)
+            host_gap(torch)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             fn()
@@ -949,7 +957,7 @@ def run_gemm_only(args, local):
     ts = []
     for i in range(args.warmup + args.steps):
         flush.zero_()
-        torch.cuda._sleep(HOST_GAP_CYCLES)
+        host_gap(torch)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         inv.comp_gemm(hi, lo, P, e, out=y)
@@ -986,7 +994,7 @@ def run_rmsnorm_only(args, local):
     ts = []
     for i in range(args.warmup + args.steps):
         flush.zero_()
-        torch.cuda._sleep(HOST_GAP_CYCLES)
+        host_gap(torch)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         inv.rmsnorm_bi(x, gamma, 1e-6, want_y=False, want_split=True)
