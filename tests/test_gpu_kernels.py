@@ -256,7 +256,10 @@ def _attn_case(inv, B, Hq, Hkv, lens, seed, max_len):
 
 @pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 4), (4, 4)])
 def test_attention_parity_edges(inv, Hq, Hkv):
-    lens = np.array([1, 2, 63, 64, 255, 256, 257, 700], np.int32)
+    # split edges (255, 256, 257) and the decode kernel's 32-key staging halves: a
+    # warp's last keys in its first half only (31, 32, 96, 160, 224, 288 = 256 + 32)
+    # or one key into its second half (33, 97)
+    lens = np.array([1, 2, 31, 32, 33, 63, 64, 96, 97, 160, 224, 255, 256, 257, 288, 700], np.int32)
     B = len(lens)
     q, oc, gc = _attn_case(inv, B, Hq, Hkv, lens, seed=30, max_len=768)
     sigma = np.float32(1 / np.sqrt(128))
