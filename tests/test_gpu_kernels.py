@@ -125,12 +125,6 @@ def test_kv_quant_bad_index_reports(inv):
 
 # ------------------------------------------------------------- comp_gemm -----
 
-def _gemm(inv, A, W):
-    P, e = inv.heal_pack_weight(dev(W))
-    hi, lo = inv.heal_split(dev(A))
-    return inv.comp_gemm(hi, lo, P, e), (P, e, hi, lo)
-
-
 def test_comp_gemm_tiny_config(inv):
     """RMSNorm(512) then the compensated GEMM K = N = 512, M = 1..8."""
     x = synth.normal((8, 512), seed=0)

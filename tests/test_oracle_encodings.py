@@ -10,7 +10,6 @@ import warnings
 from fractions import Fraction
 
 import numpy as np
-import pytest
 import torch
 
 from oracle import encodings as enc

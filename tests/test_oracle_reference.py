@@ -7,7 +7,6 @@ attention, the Hugging Face LLaMA decoder block and model).
 from fractions import Fraction
 
 import numpy as np
-import pytest
 import torch
 
 from invariant_numerics_b200 import synth
